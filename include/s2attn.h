@@ -1,0 +1,126 @@
+/*
+ * s2attn.h -- C ABI of libs2attn.so: shifted sparse attention (S²-Attn)
+ * forward and backward on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  "4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1
+ * ("S²-Attn的计算图") splits the sequence into groups of G tokens and runs
+ * causal attention inside each group.  Heads [0, H/2) use the original
+ * boundaries b(i) = floor(i/G); heads [H/2, H) shift by s = G/2 and use
+ * b'(i) = floor((i - s)/G); the shifted heads' outputs are returned at their
+ * original token positions.  Two boundary treatments of the shifted heads are
+ * described there and both are provided:
+ *   S2_STRICT        separate short first group [0, s) and last group
+ *                    [N - s, N); no key from the future is ever visible;
+ *   S2_ROLLED        the sequence is rolled left by s and grouped, with the
+ *                    in-group triangular mask of the rolled order: the last
+ *                    group is [N - s, N) followed by [0, s), so positions
+ *                    [0, s) also see [N - s, N);
+ *   S2_DENSE_CAUSAL  plain causal attention over [0, N) for every head (the
+ *                    inference graph, §2; also the "full, G = N" setting).
+ * For query row i with visible set S_i (§3, "稀疏训练与full推理之间的目标偏移"):
+ *   o_i   = sum_{j in S_i} softmax_j(scale q_i·k_j) v_j,  scale = 1/sqrt(D)
+ *   lse_i = ln sum_{j in S_i} exp(scale q_i·k_j)
+ * and the backward gives dq, dk, dv of L = sum_i dout_i·o_i with
+ *   dL/dz_ij = a_ij dout_i·(v_j - o_i),  a_ij = exp(scale q_i·k_j - lse_i).
+ *
+ * Padding (§1): when the true length n_valid is not a multiple of G the
+ * caller pads to N (a multiple of G) before calling; group boundaries are
+ * those of the padded N.  Positions >= n_valid are never visible as keys;
+ * their query rows get o = 0, lse = -inf, and receive no gradient
+ * (dq = dk = dv = 0 there).
+ *
+ * Layout.  q, k, v, o, dout, dq, dk, dv: bfloat16, [B, N, H, D], contiguous
+ * (element (b, i, h, d) at ((b*N + i)*H + h)*D + d).  lse: float32 [B, H, N].
+ * All are DEVICE pointers on the current CUDA device, 16-byte aligned.
+ * Supported on the GPU: D in {64, 128}; for S2_STRICT / S2_ROLLED, G/2 must be
+ * a multiple of 128; for S2_DENSE_CAUSAL, N a multiple of 128.  Always: H
+ * even, G even, N a multiple of G, 1 <= n_valid <= N, B*N < 2^31.
+ *
+ * Ownership and threading.  The caller owns every buffer, including the
+ * backward workspace (size from s2attn_bwd_workspace_size).  The library
+ * allocates no device memory.  Calls are asynchronous on `stream` (a
+ * cudaStream_t; NULL = the legacy default stream) and thread-safe.
+ *
+ * Errors.  Every call returns S2_OK or a negative code.  Argument, shape and
+ * support checks happen on the host before anything is enqueued; on such an
+ * error nothing was launched.  S2_ERR_CUDA reports a failed launch.  A kernel
+ * that waits on a barrier for longer than about two seconds gives up, leaves
+ * its outputs undefined and records a timeout that s2attn_check_status()
+ * reports as S2_ERR_TIMEOUT.  s2attn_last_error() returns a message for the
+ * last non-OK status of the calling thread.
+ */
+#ifndef S2ATTN_H_
+#define S2ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { S2_STRICT = 0, S2_ROLLED = 1, S2_DENSE_CAUSAL = 2 } s2_variant;
+
+enum {
+  S2_OK = 0,
+  S2_ERR_INVALID_ARG = -1, /* null or misaligned pointer, unknown enum value */
+  S2_ERR_SHAPE = -2,       /* H, G, N, n_valid violate the divisibility / range rules */
+  S2_ERR_UNSUPPORTED = -3, /* valid for the method but not for these kernels (D, G/2 % 128, GPU) */
+  S2_ERR_CUDA = -4,        /* a CUDA runtime call failed */
+  S2_ERR_TIMEOUT = -5      /* a kernel gave up waiting on a barrier */
+};
+
+/* Forward.  Writes o [B,N,H,D] (bf16) and lse [B,H,N] (fp32) for all N rows. */
+int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+               int64_t N, int64_t H, int64_t D, int64_t G, int variant, void* stream);
+
+/* Forward with a valid length n_valid <= N (the call above is n_valid = N). */
+int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                 int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                 void* stream);
+
+/* Bytes of device workspace s2attn_bwd needs: a float32 row statistic
+ * Delta_i = dout_i·o_i ([B,H,N]) and a float32 dq accumulator ([B,N,H,D]). */
+size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D);
+
+/* Backward.  Inputs q, k, v, o, dout (bf16), lse (fp32) as produced by the
+ * forward with the same B, N, H, D, G, variant (and n_valid).  Writes dq, dk,
+ * dv (bf16 [B,N,H,D]).  `workspace` must hold workspace_bytes >=
+ * s2attn_bwd_workspace_size(B, N, H, D) bytes, 256-byte aligned; its contents
+ * on entry do not matter. */
+int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H,
+               int64_t D, int64_t G, int variant, void* workspace, size_t workspace_bytes,
+               void* stream);
+
+int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H,
+                 int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace,
+                 size_t workspace_bytes, void* stream);
+
+/* Debug: the (query, key) pairs the kernels visit for one head class
+ * (0: heads [0,H/2), 1: heads [H/2,H); ignored for S2_DENSE_CAUSAL), computed
+ * by the same scheduler and masks as the forward/backward kernels.
+ *   format 0: bitset, uint32 [N][ceil(N/32)], bit j of row i set iff key j is
+ *             visited from query i (N <= 65536);
+ *   format 1: int32 [N][4] = {lo1, hi1, lo2, hi2}, the visited keys as at most
+ *             two inclusive intervals of original positions, -1 when absent.
+ * `out` is a device pointer the caller sized accordingly. */
+int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                           int format, void* out, void* stream);
+
+/* Synchronizes `stream` and reports (then clears) a kernel timeout recorded
+ * on the current device since the last check: S2_OK or S2_ERR_TIMEOUT. */
+int s2attn_check_status(void* stream);
+
+/* Message for the last non-OK status returned to the calling thread. */
+const char* s2attn_last_error(void);
+
+/* ABI version of this header (major*100 + minor). */
+int s2attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2ATTN_H_ */

@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
         L.s2o_visible.restype = ctypes.c_int
         L.s2o_adjacency.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int, u8p]
         L.s2o_adjacency.restype = None
+        L.s2o_adjacency_row.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int, i64, u8p]
+        L.s2o_adjacency_row.restype = None
         L.s2o_pair_count.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
         L.s2o_pair_count.restype = i64
         L.s2o_attention.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, i64,
@@ -89,6 +91,13 @@ def adjacency(N: int, G: int, n_valid: int, variant: int, head_class: int) -> np
     """Explicit boolean matrix A^(head_class) of shape [N, N] (row i = query)."""
     out = np.zeros((N, N), dtype=np.uint8)
     lib().s2o_adjacency(N, G, n_valid, variant, head_class, _ptr(out, ctypes.c_uint8))
+    return out.astype(bool)
+
+
+def adjacency_row(N: int, G: int, n_valid: int, variant: int, head_class: int, i: int) -> np.ndarray:
+    """Row i of A^(head_class) as a boolean vector of length N."""
+    out = np.zeros(N, dtype=np.uint8)
+    lib().s2o_adjacency_row(N, G, n_valid, variant, head_class, i, _ptr(out, ctypes.c_uint8))
     return out.astype(bool)
 
 

@@ -88,6 +88,12 @@ void s2o_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_
       out[i * N + j] = (uint8_t)s2o_visible(N, G, n_valid, variant, head_class, i, j);
 }
 
+/* One row of A: out[j] = A[i][j] for j in [0, N). */
+void s2o_adjacency_row(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class, int64_t i,
+                       uint8_t* out) {
+  for (int64_t j = 0; j < N; ++j) out[j] = (uint8_t)s2o_visible(N, G, n_valid, variant, head_class, i, j);
+}
+
 /* Number of visible (i, j) pairs, by enumeration. */
 int64_t s2o_pair_count(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class) {
   int64_t c = 0;

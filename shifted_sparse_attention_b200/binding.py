@@ -1,0 +1,192 @@
+"""Thin ctypes binding of libs2attn.so (declared in include/s2attn.h).
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  PyTorch supplies device memory and the current
+stream.  There is no fallback: if the library is missing or the GPU is not an
+sm_100a part, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import torch
+
+STRICT, ROLLED, DENSE_CAUSAL = 0, 1, 2
+S2_OK, S2_ERR_INVALID_ARG, S2_ERR_SHAPE, S2_ERR_UNSUPPORTED, S2_ERR_CUDA, S2_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+
+LIB_PATH = Path(__file__).resolve().parent / "libs2attn.so"
+
+# name -> (argtypes, restype), mirroring include/s2attn.h
+_i64, _int, _vp, _fp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+SIGNATURES = {
+    "s2attn_fwd": ([_vp, _vp, _vp, _vp, _fp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
+    "s2attn_fwd_v": ([_vp, _vp, _vp, _vp, _fp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
+    "s2attn_bwd_workspace_size": ([_i64, _i64, _i64, _i64], _sz),
+    "s2attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int,
+                    _vp, _sz, _vp], _int),
+    "s2attn_bwd_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
+                      _int, _vp, _sz, _vp], _int),
+    "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
+    "s2attn_check_status": ([_vp], _int),
+    "s2attn_last_error": ([], ctypes.c_char_p),
+    "s2attn_version": ([], _int),
+}
+
+_lib = None
+
+
+class S2AttnError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__("s2attn error %d: %s" % (code, message))
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libs2attn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise ImportError("libs2attn.so is not built; run `python -m shifted_sparse_attention_b200.build`")
+        L = ctypes.CDLL(str(LIB_PATH))
+        for name, (args, res) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != S2_OK:
+        raise S2AttnError(rc, lib().s2attn_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ------------------------------------------------------------------ raw entry points (same names as the C ABI)
+
+
+def s2attn_fwd_v(q, k, v, o, lse, B, N, H, D, G, n_valid, variant, stream=None) -> int:
+    return lib().s2attn_fwd_v(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, N, H, D, G, n_valid, variant,
+                              _stream(stream))
+
+
+def s2attn_fwd(q, k, v, o, lse, B, N, H, D, G, variant, stream=None) -> int:
+    return lib().s2attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, N, H, D, G, variant, _stream(stream))
+
+
+def s2attn_bwd_workspace_size(B, N, H, D) -> int:
+    return int(lib().s2attn_bwd_workspace_size(B, N, H, D))
+
+
+def s2attn_bwd_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace, workspace_bytes,
+                 stream=None) -> int:
+    return lib().s2attn_bwd_v(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                              _ptr(dv), B, N, H, D, G, n_valid, variant, _ptr(workspace), workspace_bytes,
+                              _stream(stream))
+
+
+def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, variant, workspace, workspace_bytes,
+               stream=None) -> int:
+    return lib().s2attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                            _ptr(dv), B, N, H, D, G, variant, _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, out, stream=None) -> int:
+    return lib().s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, _ptr(out), _stream(stream))
+
+
+def s2attn_check_status(stream=None) -> int:
+    return lib().s2attn_check_status(_stream(stream))
+
+
+def s2attn_last_error() -> str:
+    return lib().s2attn_last_error().decode()
+
+
+# ------------------------------------------------------------------ tensor-level helpers
+
+
+def _shape(q):
+    if q.dim() != 4 or q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+        raise ValueError("expected a contiguous CUDA bf16 tensor [B, N, H, D]")
+    return tuple(int(x) for x in q.shape)
+
+
+def forward(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None, out=None, lse=None, stream=None):
+    """S²-Attn forward; returns (o [B,N,H,D] bf16, lse [B,H,N] fp32)."""
+    B, N, H, D = _shape(q)
+    nv = N if n_valid is None else int(n_valid)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(s2attn_fwd_v(q, k, v, o, l, B, N, H, D, G, nv, variant, stream))
+    return o, l
+
+
+def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int | None = None,
+             grads=None, workspace=None, stream=None):
+    """S²-Attn backward; returns (dq, dk, dv) bf16 [B,N,H,D]."""
+    B, N, H, D = _shape(q)
+    nv = N if n_valid is None else int(n_valid)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = grads
+    ws_bytes = s2attn_bwd_workspace_size(B, N, H, D)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    _check(s2attn_bwd_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, nv, variant, workspace,
+                        workspace.numel() * workspace.element_size(), stream))
+    return dq, dk, dv
+
+
+def debug_adjacency(N: int, G: int, variant: int, head_class: int, n_valid: int | None = None,
+                    fmt: int = 0, device="cuda"):
+    """Visited (query, key) pattern of one head class, from the kernels' scheduler."""
+    nv = N if n_valid is None else int(n_valid)
+    if fmt == 0:
+        out = torch.empty((N, (N + 31) // 32), dtype=torch.int32, device=device)
+    else:
+        out = torch.empty((N, 4), dtype=torch.int32, device=device)
+    _check(s2attn_debug_adjacency(N, G, nv, variant, head_class, fmt, out))
+    return out
+
+
+def check_status(stream=None) -> None:
+    _check(s2attn_check_status(stream))
+
+
+class S2Attention(torch.autograd.Function):
+    """Autograd wrapper: forward and backward both run in libs2attn.so."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, G, variant=STRICT, n_valid=None):
+        o, lse = forward(q, k, v, G, variant, n_valid)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.cfg = (G, variant, n_valid)
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        G, variant, n_valid = ctx.cfg
+        dq, dk, dv = backward(q, k, v, o, do.contiguous(), lse, G, variant, n_valid)
+        return dq, dk, dv, None, None, None
+
+
+def s2_attention(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None):
+    return S2Attention.apply(q, k, v, G, variant, n_valid)

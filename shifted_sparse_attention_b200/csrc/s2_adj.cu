@@ -1,0 +1,75 @@
+// s2_adj.cu -- debug dump of the visibility pattern the kernels actually use.
+//
+// Walks the same work-unit decomposition (decode_unit), the same key-tile
+// list (ktile_valid / tile_takes) and the same per-row column limits
+// (col_limit) as the forward and backward kernels, and writes, for every
+// query row of one head class, the set of keys those kernels visit, in
+// original positions.  Comparing it bit for bit with the explicit matrices
+// A^(0) / A^(1) of "4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1 checks the
+// scheduler and the masks independently of any floating-point result.
+#include <cuda_runtime.h>
+
+#include "s2_index.cuh"
+#include "s2_kernels.h"
+
+namespace s2 {
+
+// One CTA per work unit of a head of class `cls`; thread = one row of the
+// unit's two query tiles.
+__global__ void __launch_bounds__(256) s2_adjacency_kernel(const Plan p, int cls, int format,
+                                                           uint32_t* __restrict__ bits,
+                                                           int* __restrict__ intervals) {
+  Unit u;
+  if (!decode_unit(p, blockIdx.x, u)) return;
+  if (u.h != cls) return;  // with H = 2, head h has class h (dense: only head 0 is dumped)
+  const int x = threadIdx.x / kTile, r = threadIdx.x % kTile;
+  if (u.t[x] < 0) return;
+  const int row = tile_orig(p, u, u.t[x]) + r;
+  const int words = (p.N + 31) / 32;
+  if (format == 0)
+    for (int w = 0; w < words; ++w) bits[(size_t)row * words + w] = 0u;
+  int iv[4] = {-1, -1, -1, -1};
+  int nint = 0;
+  for (int k = 0; k <= u.t[x]; ++k) {
+    if (!tile_takes(p, u, x, k) || !ktile_valid(p, u, k)) continue;
+    const int lim = col_limit(p, u, u.t[x], k, r);
+    if (lim <= 0) continue;
+    const int lo = tile_orig(p, u, k), hi = lo + lim - 1;
+    if (format == 0) {
+      for (int j = lo; j <= hi; ++j) bits[(size_t)row * words + j / 32] |= 1u << (j % 32);
+    } else {
+      if (nint > 0 && iv[2 * (nint - 1) + 1] + 1 == lo) {
+        iv[2 * (nint - 1) + 1] = hi;
+      } else if (nint < 2) {
+        iv[2 * nint] = lo;
+        iv[2 * nint + 1] = hi;
+        ++nint;
+      } else {
+        iv[0] = iv[1] = iv[2] = iv[3] = -2;  // more than two intervals: never expected
+      }
+    }
+  }
+  if (format == 1)
+    for (int c = 0; c < 4; ++c) intervals[(size_t)row * 4 + c] = iv[c];
+}
+
+__global__ void s2_fill_kernel(int* out, size_t n, int value) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    out[i] = value;
+}
+
+int launch_adjacency(const Plan& p0, int head_class, int format, void* out, cudaStream_t stream) {
+  // A head of each class: with H = 2, head 0 is class 0 and head 1 is class 1.
+  Plan p = p0;
+  p.B = 1;
+  p.H = 2;
+  // rows that no tile covers cannot exist, but start from a defined state
+  if (format == 1)
+    s2_fill_kernel<<<64, 256, 0, stream>>>(static_cast<int*>(out), (size_t)p.N * 4, -1);
+  const int grid = p.ranks * 2;
+  s2_adjacency_kernel<<<grid, 256, 0, stream>>>(p, head_class, format, static_cast<uint32_t*>(out),
+                                                static_cast<int*>(out));
+  return (int)cudaGetLastError();
+}
+
+}  // namespace s2

@@ -1,0 +1,397 @@
+// s2_fwd.cu -- S²-Attn forward on sm_100a (tcgen05 tensor cores, TMA, TMEM).
+//
+// Computes, per head and query row i with visible set S_i
+// ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调", §3):
+//     o_i = sum_{j in S_i} softmax_j(q_i·k_j / sqrt(D)) v_j,
+//     lse_i = ln sum_{j in S_i} exp(q_i·k_j / sqrt(D)),
+// where S_i is the causal part of i's group (§1, see s2_index.cuh).
+// Only key tiles of i's own segment up to the diagonal are visited: no
+// off-group tile is ever loaded or multiplied, so the work is O(N·G).
+//
+// CTA = two consecutive 128-row query tiles (A, B) of one segment sharing
+// every K/V tile.  Warp roles (320 threads):
+//   warps 0-3  softmax of tile A (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax of tile B
+//   warp  8    TMA producer: Q tiles once, then the K/V stream
+//   warp  9    TMEM allocator and tcgen05.mma issuer (one thread)
+// TMEM (512 columns): S_A [0,128), S_B [128,256), O_A and O_B at 256 + x·D.
+// Shared memory: Q_A, Q_B, a ring of three K/V slots, P_A, P_B; all tiles
+// are 128-byte-swizzled, 1024-byte aligned, as TMA writes and UMMA reads them.
+// MMA order per key tile k (software pipelined so that the tensor core works
+// on the next S while the softmax warps exponentiate the current one):
+//     S_A(k+1)=Q_A K(k+1)^T, O_A += P_A(k) V(k), S_B(k+1)=Q_B K(k+1)^T, O_B += P_B(k) V(k)
+// Softmax uses base-2 exponentials with a lazily updated running max: O and
+// l are rescaled only when the row max grows by more than 8 (a factor 256),
+// which keeps bf16 P and fp32 sums exact enough and skips most rescales.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "s2_index.cuh"
+#include "s2_kernels.h"
+#include "sm100_ptx.cuh"
+
+namespace s2 {
+
+namespace fwd {
+
+constexpr int kThreads = 320;
+constexpr int kSlots = 3;
+constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 = one 128B-swizzle column block
+
+enum Bar {
+  KV_FULL = 0,      // + slot (3)
+  KV_EMPTY = 3,     // + slot (3)
+  S_FULL = 6,       // + tile (2)
+  S_FREE = 8,       // + tile (2)
+  P_FULL = 10,      // + tile (2)
+  PV_DONE = 12,     // + tile (2)
+  Q_FULL = 14,
+  MMA_DONE = 15,
+  NUM_BARS = 16
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kQBytes = kTile * D * 2;
+  static constexpr int kKVBytes = kTile * D * 2;
+  static constexpr int kPBytes = kTile * kTile * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kKV = 2 * kQBytes;
+  static constexpr int kP = kKV + kSlots * kKVBytes;
+  static constexpr int kBars = kP + 2 * kPBytes;
+  static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+};
+
+// Smallest valid key tile > k (and <= kmax), or -1.
+__device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k) {
+  for (int j = k + 1; j <= u.kmax; ++j)
+    if (ktile_valid(p, u, j)) return j;
+  return -1;
+}
+
+}  // namespace fwd
+
+template <int D>
+__global__ void __launch_bounds__(fwd::kThreads, 1)
+    s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const Plan p, float* __restrict__ lse, int* __restrict__ status) {
+  using namespace fwd;
+  using L = Layout<D>;
+  constexpr int kChunks = D / 64;
+
+  Unit u;
+  if (!decode_unit(p, blockIdx.x, u)) return;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  auto sQ = [&](int x) { return sb + L::kQ + x * L::kQBytes; };
+  auto sKV = [&](int slot) { return sb + L::kKV + slot * L::kKVBytes; };
+  auto sP = [&](int x) { return sb + L::kP + x * L::kPBytes; };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(bar(KV_FULL + i), 1);
+      mbar_init(bar(KV_EMPTY + i), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(S_FULL + x), 1);
+      mbar_init(bar(S_FREE + x), 128);
+      mbar_init(bar(P_FULL + x), 128);
+      mbar_init(bar(PV_DONE + x), 1);
+    }
+    mbar_init(bar(Q_FULL), 1);
+    mbar_init(bar(MMA_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int row_base = u.b * p.N;  // TMA outer coordinate of position 0 of this batch row
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && u.kmax >= 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      uint32_t qbytes = 0;
+      for (int x = 0; x < 2; ++x) qbytes += u.part[x] ? L::kQBytes : 0;
+      mbar_arrive_expect_tx(bar(Q_FULL), qbytes);
+      for (int x = 0; x < 2; ++x) {
+        if (!u.part[x]) continue;
+        const int row = row_base + tile_orig(p, u, u.t[x]);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(sQ(x) + c * kChunkBytes, &tmQ, c * 64, u.h, row, bar(Q_FULL));
+      }
+      int e = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap* tm, int k) {
+        const int slot = e % kSlots;
+        if (e >= kSlots) ok = s2_wait(bar(KV_EMPTY + slot), ((e / kSlots) - 1) & 1, abort_flag, status, 1);
+        if (!ok) return;
+        mbar_arrive_expect_tx(bar(KV_FULL + slot), L::kKVBytes);
+        const int row = row_base + tile_orig(p, u, k);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(sKV(slot) + c * kChunkBytes, tm, c * 64, u.h, row, bar(KV_FULL + slot));
+        ++e;
+      };
+      int kc = next_k(p, u, -1);
+      if (kc >= 0) load(&tmK, kc);
+      while (ok && kc >= 0) {
+        const int kn = next_k(p, u, kc);
+        if (kn >= 0) load(&tmK, kn);
+        if (!ok) break;
+        load(&tmV, kc);
+        kc = kn;
+      }
+      // drain: the last loads must land before the CTA retires
+      for (int d = (e > kSlots ? e - kSlots : 0); d < e; ++d)
+        s2_wait(bar(KV_FULL + d % kSlots), (d / kSlots) & 1, abort_flag, status, 1);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && u.kmax >= 0) {
+      constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
+      auto issue_qk = [&](int x, int slot) {
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
+          umma_ss(tmem + x * 128, umma_desc_sw128(sQ(x) + off, 16, 1024),
+                  umma_desc_sw128(sKV(slot) + off, 16, 1024), idesc_qk, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int x, int slot, bool acc) {
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          const uint32_t aoff = (kk / 4) * kChunkBytes + (kk % 4) * 32;
+          umma_ss(tmem + 256 + x * D, umma_desc_sw128(sP(x) + aoff, 16, 1024),
+                  umma_desc_sw128(sKV(slot) + kk * 2048, kChunkBytes, 1024), idesc_pv,
+                  (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
+      int nqk[2] = {0, 0}, npv[2] = {0, 0};
+      int e = 0;
+      int kc = next_k(p, u, -1);
+      if (ok && kc >= 0) {
+        const int eK = e++;
+        ok = s2_wait(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
+        tc_fence_after();
+        for (int x = 0; ok && x < 2; ++x)
+          if (tile_takes(p, u, x, kc)) {
+            issue_qk(x, eK % kSlots);
+            umma_commit(bar(S_FULL + x));
+            ++nqk[x];
+          }
+        umma_commit(bar(KV_EMPTY + eK % kSlots));
+      }
+      while (ok && kc >= 0) {
+        const int kn = next_k(p, u, kc);
+        const int eK = (kn >= 0) ? e++ : -1;
+        const int eV = e++;
+        if (kn >= 0) {
+          ok = s2_wait(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        for (int x = 0; x < 2; ++x) {
+          if (kn >= 0 && tile_takes(p, u, x, kn)) {
+            if (nqk[x] > 0) ok = s2_wait(bar(S_FREE + x), (nqk[x] - 1) & 1, abort_flag, status, 2);
+            if (!ok) break;
+            tc_fence_after();
+            issue_qk(x, eK % kSlots);
+            umma_commit(bar(S_FULL + x));
+            ++nqk[x];
+          }
+          if (x == 1 && kn >= 0) umma_commit(bar(KV_EMPTY + eK % kSlots));
+          if (tile_takes(p, u, x, kc)) {
+            if (x == 0 || !tile_takes(p, u, 0, kc)) {
+              ok = s2_wait(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
+              if (!ok) break;
+            }
+            ok = s2_wait(bar(P_FULL + x), npv[x] & 1, abort_flag, status, 2);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(x, eV % kSlots, npv[x] > 0);
+            umma_commit(bar(PV_DONE + x));
+            ++npv[x];
+          }
+        }
+        if (!ok) break;
+        umma_commit(bar(KV_EMPTY + eV % kSlots));
+        kc = kn;
+      }
+      // every issued MMA must be complete before TMEM is released
+      umma_commit(bar(MMA_DONE));
+      s2_wait(bar(MMA_DONE), 0, abort_flag, status, 2);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int x = warp / 4;
+    const int wq = warp % 4;
+    const int r = wq * 32 + lane;  // row within the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + x * 128;
+    const uint32_t tO = tmem + lane_off + 256 + x * D;
+    if (u.t[x] >= 0) {
+      const int q0 = tile_orig(p, u, u.t[x]);
+      const bool row_valid = (q0 + r) < p.n_valid;
+      float m_used = -INFINITY, l = 0.f;
+      int n = 0;
+      bool ok = true;
+      if (u.part[x]) {
+        for (int k = 0; k <= u.t[x] && ok; ++k) {
+          if (!ktile_valid(p, u, k)) continue;
+          ok = s2_wait(bar(S_FULL + x), n & 1, abort_flag, status, 4);
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t s[kTile];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[j * 32]));
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(bar(S_FREE + x));
+
+          const int lim = col_limit(p, u, u.t[x], k, r);
+          float mx = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < kTile; ++c)
+            if (c < lim) mx = fmaxf(mx, __uint_as_float(s[c]) * p.scale_log2);
+          const float m_new = fmaxf(m_used, mx);
+          const bool need = m_new > m_used + 8.0f;
+          float factor = 1.f;
+          if (need) {
+            factor = ex2(m_used - m_new);  // 0 when m_used = -inf
+            l *= factor;
+            m_used = m_new;
+          }
+          const float m_exp = (m_used == -INFINITY) ? 0.f : m_used;
+          // p = 2^(x - m), rounded to bf16 pairs in place (s[c/2] <- pair c, c+1);
+          // l sums the ROUNDED weights, so o = sum p~ v / sum p~ stays a convex
+          // combination of the v_j whatever the rounding of each p.
+          float sum = 0.f;
+#pragma unroll
+          for (int c = 0; c < kTile; c += 2) {
+            const float e0 = (c < lim) ? ex2(fmaf(__uint_as_float(s[c]), p.scale_log2, -m_exp)) : 0.f;
+            const float e1 = (c + 1 < lim) ? ex2(fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -m_exp)) : 0.f;
+            const uint32_t pk = pack_bf16(e0, e1);
+            s[c / 2] = pk;
+            sum += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+          }
+          l += sum;
+
+          if (n > 0) {
+            ok = s2_wait(bar(PV_DONE + x), (n - 1) & 1, abort_flag, status, 4);
+            if (!ok) break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, need)) {
+              const float f = need ? factor : 1.f;
+#pragma unroll
+              for (int j = 0; j < D / 32; ++j) {
+                uint32_t o[32];
+                tmem_ld32(tO + j * 32, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+                tmem_st32(tO + j * 32, o);
+              }
+              tmem_wait_st();
+            }
+          }
+          // P (bf16) -> shared memory, K-major, 128B swizzle
+#pragma unroll
+          for (int pc = 0; pc < 16; ++pc) {
+            const uint32_t addr = sP(x) + (pc / 8) * kChunkBytes + r * 128 + (((pc % 8) ^ (r & 7)) << 4);
+            st_shared_v4(addr, s[pc * 4], s[pc * 4 + 1], s[pc * 4 + 2], s[pc * 4 + 3]);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          mbar_arrive(bar(P_FULL + x));
+          ++n;
+        }
+        if (ok && n > 0) {
+          ok = s2_wait(bar(PV_DONE + x), (n - 1) & 1, abort_flag, status, 4);
+          tc_fence_after();
+        }
+      }
+      // ---------------------------------------------------------- epilogue
+      const bool have = u.part[x] && ok && n > 0;
+      const float inv_l = (have && row_valid) ? 1.f / l : 0.f;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t o[32];
+        if (have) {
+          tmem_ld32(tO + j * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+#pragma unroll
+        for (int pc = 0; pc < 4; ++pc) {
+          const int col = j * 32 + pc * 8;  // first of 8 columns
+          const int chunk = col / 64, piece = (col % 64) / 8;
+          const uint32_t addr = sP(x) + chunk * kChunkBytes + r * 128 + ((piece ^ (r & 7)) << 4);
+          const uint32_t* oo = &o[pc * 8];
+          st_shared_v4(addr, pack_bf16(__uint_as_float(oo[0]) * inv_l, __uint_as_float(oo[1]) * inv_l),
+                       pack_bf16(__uint_as_float(oo[2]) * inv_l, __uint_as_float(oo[3]) * inv_l),
+                       pack_bf16(__uint_as_float(oo[4]) * inv_l, __uint_as_float(oo[5]) * inv_l),
+                       pack_bf16(__uint_as_float(oo[6]) * inv_l, __uint_as_float(oo[7]) * inv_l));
+        }
+      }
+      const float lse_v = (have && row_valid) ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      lse[((size_t)u.b * p.H + u.h) * p.N + q0 + r] = lse_v;
+      fence_proxy_async_smem();
+      named_bar_sync(1 + x, 128);
+      if (r == 0) {
+        for (int c = 0; c < kChunks; ++c)
+          tma_store_3d(&tmO, sP(x) + c * kChunkBytes, c * 64, u.h, row_base + q0);
+        tma_store_commit();
+        tma_store_wait_all();
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+int launch_fwd_impl(const FwdArgs& a) {
+  using L = fwd::Layout<D>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  if (e != cudaSuccess) return (int)e;
+  const int grid = a.plan.ranks * a.plan.B * a.plan.H;
+  s2_fwd_kernel<D><<<grid, fwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmO, a.plan,
+                                                                 a.lse, a.status);
+  return (int)cudaGetLastError();
+}
+
+int launch_fwd(const FwdArgs& a) {
+  if (a.plan.D == 64) return launch_fwd_impl<64>(a);
+  return launch_fwd_impl<128>(a);
+}
+
+}  // namespace s2

@@ -1,0 +1,181 @@
+// s2_index.cuh -- S²-Attn segment / tile scheduler and mask predicates,
+// shared by the host launcher and every kernel (forward, backward, adjacency
+// dump), so that all of them visit exactly the same (query, key) pairs.
+//
+// Method ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调", §1 "S²-Attn的计算图"):
+//   heads [0, H/2) group positions by b(i) = floor(i/G); heads [H/2, H) shift
+//   by s = G/2 and group by b'(i) = floor((i - s)/G); attention is causal
+//   inside a group; the shifted heads' outputs go back to original positions.
+//   Boundary variants of the shifted heads (same section):
+//     STRICT  -- separate short head group [0, s) and tail group [N - s, N);
+//     ROLLED  -- roll left by s and keep the in-group triangular mask, so the
+//                last group is [N - s, N) followed by [0, s);
+//   DENSE_CAUSAL is the full causal graph used at inference (§2).
+//   The reshape [B, N, H, D] -> [B*M, G, H, D] of §1 becomes index math here:
+//   no tensor is ever rolled or copied.
+//
+// Virtual coordinates.  For every (head class, variant) the rows of a head
+// are laid out in a "virtual" order in which each segment is a contiguous
+// range and causality is "virtual key <= virtual query":
+//   class 0, STRICT class 1, DENSE: virtual index = original position;
+//   ROLLED class 1: virtual index r = rolled position, original = (r + s) mod N.
+// With s a multiple of 128, every 128-row tile of virtual rows is a
+// contiguous range of original positions, so each tile is one TMA box.
+#pragma once
+#include <cstdint>
+
+#ifdef __CUDACC__
+#define S2_HD __host__ __device__ __forceinline__
+#else
+#define S2_HD inline
+#endif
+
+namespace s2 {
+
+constexpr int kTile = 128;  // rows per query tile and per key tile
+
+enum Variant { kStrict = 0, kRolled = 1, kDenseCausal = 2 };
+
+struct Plan {
+  int B, N, H, D, G, s, n_valid, variant;
+  int nseg[2];     // segments per head class
+  int nunit[2];    // max work units (pairs of q tiles) per segment, per class
+  int ranks;       // max over classes of nseg * nunit
+  float scale_log2;  // log2(e) / sqrt(D)
+};
+
+S2_HD int head_class(const Plan& p, int h) {
+  return (p.variant == kDenseCausal) ? 0 : (h >= p.H / 2 ? 1 : 0);
+}
+
+S2_HD int seg_count(const Plan& p, int cls) {
+  if (p.variant == kDenseCausal) return 1;
+  if (cls == 1 && p.variant == kStrict) return p.N / p.G + 1;
+  return p.N / p.G;
+}
+
+// Virtual range [vbeg, vbeg + len) of segment `seg`.
+S2_HD void seg_bounds(const Plan& p, int cls, int seg, int& vbeg, int& len) {
+  if (p.variant == kDenseCausal) { vbeg = 0; len = p.N; return; }
+  if (cls == 1 && p.variant == kStrict) {
+    const int M = p.N / p.G;
+    if (seg == 0) { vbeg = 0; len = p.s; return; }
+    if (seg == M) { vbeg = p.N - p.s; len = p.s; return; }
+    vbeg = p.s + (seg - 1) * p.G; len = p.G; return;
+  }
+  vbeg = seg * p.G; len = p.G;
+}
+
+// Segment containing virtual row v.
+S2_HD int seg_of(const Plan& p, int cls, int v) {
+  if (p.variant == kDenseCausal) return 0;
+  if (cls == 1 && p.variant == kStrict) {
+    if (v < p.s) return 0;
+    const int M = p.N / p.G;
+    if (v >= p.N - p.s) return M;
+    return (v - p.s) / p.G + 1;
+  }
+  return v / p.G;
+}
+
+S2_HD int orig_of(const Plan& p, int cls, int v) {
+  if (cls == 1 && p.variant == kRolled) {
+    int o = v + p.s;
+    return o >= p.N ? o - p.N : o;
+  }
+  return v;
+}
+
+S2_HD int virt_of(const Plan& p, int cls, int x) {
+  if (cls == 1 && p.variant == kRolled) {
+    int v = x - p.s;
+    return v < 0 ? v + p.N : v;
+  }
+  return x;
+}
+
+// One CTA work unit: up to two consecutive query tiles of one segment.
+struct Unit {
+  int b, h, cls;
+  int vbeg;        // virtual start of the segment
+  int ntiles;      // query tiles in the segment
+  int t[2];        // local tile indices (t[1] = -1 if absent)
+  bool part[2];    // tile exists and holds at least one valid row
+  int kmax;        // largest key tile index any participating tile needs (-1: none)
+};
+
+// Original position of the first row of local tile `t` of the unit's segment.
+S2_HD int tile_orig(const Plan& p, const Unit& u, int t) {
+  return orig_of(p, u.cls, u.vbeg + t * kTile);
+}
+
+// Decode a linear work index (longest work first).  Returns false for idle indices.
+S2_HD bool decode_unit(const Plan& p, int L, Unit& u) {
+  const int BH = p.B * p.H;
+  const int bh = L % BH, r = L / BH;
+  u.b = bh / p.H;
+  u.h = bh % p.H;
+  u.cls = head_class(p, u.h);
+  const int S = p.nseg[u.cls], NU = p.nunit[u.cls];
+  if (r >= S * NU) return false;
+  const int unit = NU - 1 - r / S;
+  const int seg = r % S;
+  int len;
+  seg_bounds(p, u.cls, seg, u.vbeg, len);
+  u.ntiles = len / kTile;
+  if (2 * unit >= u.ntiles) return false;
+  u.t[0] = 2 * unit;
+  u.t[1] = (2 * unit + 1 < u.ntiles) ? 2 * unit + 1 : -1;
+  u.kmax = -1;
+  for (int x = 0; x < 2; ++x) {
+    u.part[x] = (u.t[x] >= 0) && (tile_orig(p, u, u.t[x]) < p.n_valid);
+    if (u.part[x]) u.kmax = u.t[x];
+  }
+  return true;
+}
+
+// A key tile is processed iff it holds at least one valid key.
+S2_HD bool ktile_valid(const Plan& p, const Unit& u, int k) {
+  return tile_orig(p, u, k) < p.n_valid;
+}
+
+// Query tile x takes part at key tile k.
+S2_HD bool tile_takes(const Plan& p, const Unit& u, int x, int k) {
+  return u.part[x] && k <= u.t[x];
+}
+
+// Number of key columns of key tile k visible from local row r (0..127) of
+// query tile tq: columns [0, limit) are visible, the rest masked.  Combines
+// the causal triangle of the diagonal tile with the padding mask on keys and
+// on the query row (positions >= n_valid).
+S2_HD int col_limit(const Plan& p, const Unit& u, int tq, int k, int r) {
+  const int q0 = tile_orig(p, u, tq);
+  if (q0 + r >= p.n_valid) return 0;
+  int lim = (k == tq) ? r + 1 : kTile;
+  const int kv = p.n_valid - tile_orig(p, u, k);
+  return lim < kv ? lim : kv;
+}
+
+// Host-side plan construction (validated by the caller).
+inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int variant) {
+  Plan p{};
+  p.B = B; p.N = N; p.H = H; p.D = D; p.G = G; p.s = G / 2;
+  p.n_valid = n_valid; p.variant = variant;
+  for (int c = 0; c < 2; ++c) {
+    p.nseg[c] = seg_count(p, c);
+    int maxlen = 0;
+    for (int sgi = 0; sgi < p.nseg[c]; ++sgi) {
+      int vb, len;
+      seg_bounds(p, c, sgi, vb, len);
+      if (len > maxlen) maxlen = len;
+    }
+    const int nt = maxlen / kTile;
+    p.nunit[c] = (nt + 1) / 2;
+  }
+  const int r0 = p.nseg[0] * p.nunit[0], r1 = p.nseg[1] * p.nunit[1];
+  p.ranks = r0 > r1 ? r0 : r1;
+  p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
+  return p;
+}
+
+}  // namespace s2

@@ -1,0 +1,44 @@
+// s2_kernels.h -- internal launch interface between the C-ABI layer and the
+// kernels (not installed; the public interface is include/s2attn.h).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "s2_index.cuh"
+
+namespace s2 {
+
+struct FwdArgs {
+  const CUtensorMap* tmQ;
+  const CUtensorMap* tmK;
+  const CUtensorMap* tmV;
+  const CUtensorMap* tmO;
+  Plan plan;
+  float* lse;
+  int* status;
+  cudaStream_t stream;
+};
+
+struct BwdArgs {
+  const CUtensorMap* tmQ;
+  const CUtensorMap* tmK;
+  const CUtensorMap* tmV;
+  const CUtensorMap* tmdO;
+  const CUtensorMap* tmdK;
+  const CUtensorMap* tmdV;
+  Plan plan;
+  const void* o;      // bf16 [B, N, H, D]
+  const void* dout;   // bf16 [B, N, H, D]
+  const float* lse;   // [B, H, N]
+  float* delta;       // workspace [B, H, N]
+  float* dq_acc;      // workspace [B, N, H, D] fp32
+  void* dq;           // bf16 [B, N, H, D]
+  int* status;
+  cudaStream_t stream;
+};
+
+int launch_fwd(const FwdArgs& a);
+int launch_bwd(const BwdArgs& a);
+int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
+
+}  // namespace s2

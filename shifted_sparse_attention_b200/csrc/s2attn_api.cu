@@ -1,0 +1,254 @@
+// s2attn_api.cu -- the C ABI declared in include/s2attn.h: argument and shape
+// validation (divisibility rules of "4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调"
+// §1: H even, G even, N a multiple of G; padding carried as n_valid), TMA
+// tensor-map encoding, and kernel launches.  No device memory is allocated
+// here; the only mutable state is a per-device cache (capability check,
+// timeout status word address, driver entry point).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "../../include/s2attn.h"
+#include "s2_index.cuh"
+#include "s2_kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+// Timeout / abort status word written by the kernels (bit flags per role).
+__device__ int g_s2_status;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceState {
+  bool ready = false;
+  bool supported = false;
+  int* status = nullptr;
+  EncodeTiledFn encode = nullptr;
+  std::string why;
+};
+
+constexpr int kMaxDevices = 64;
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+// Per-device set-up on first use: capability check and the status word address.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(S2_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& st = g_dev[dev];
+  if (!st.ready) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetDeviceProperties: %s", cudaGetErrorString(e));
+    if (prop.major != 10 || prop.minor != 0) {
+      st.supported = false;
+      st.why = "kernels are built for sm_100a (B200); device is sm_" + std::to_string(prop.major) +
+               std::to_string(prop.minor);
+    } else {
+      void* sym = nullptr;
+      e = cudaGetSymbolAddress(&sym, g_s2_status);
+      if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+      st.status = static_cast<int*>(sym);
+      cudaDriverEntryPointQueryResult q;
+      void* fn = nullptr;
+      e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+      if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return fail(S2_ERR_CUDA, "driver entry point cuTensorMapEncodeTiled unavailable");
+      st.encode = reinterpret_cast<EncodeTiledFn>(fn);
+      st.supported = true;
+    }
+    st.ready = true;
+  }
+  if (!st.supported) return fail(S2_ERR_UNSUPPORTED, "%s", st.why.c_str());
+  *out = &st;
+  return S2_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape rules of the method plus the kernels' own support limits.
+int validate(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant) {
+  if (variant < S2_STRICT || variant > S2_DENSE_CAUSAL)
+    return fail(S2_ERR_INVALID_ARG, "unknown variant %d", variant);
+  if (B < 1 || N < 1 || H < 1 || D < 1 || G < 1)
+    return fail(S2_ERR_SHAPE, "B, N, H, D, G must be positive (B=%lld N=%lld H=%lld D=%lld G=%lld)",
+                (long long)B, (long long)N, (long long)H, (long long)D, (long long)G);
+  if (H % 2) return fail(S2_ERR_SHAPE, "H=%lld must be even (half the heads are shifted)", (long long)H);
+  if (G % 2) return fail(S2_ERR_SHAPE, "G=%lld must be even (shift G/2)", (long long)G);
+  if (N % G) return fail(S2_ERR_SHAPE, "N=%lld must be a multiple of G=%lld (pad first)", (long long)N, (long long)G);
+  if (n_valid < 1 || n_valid > N)
+    return fail(S2_ERR_SHAPE, "n_valid=%lld must be in [1, N=%lld]", (long long)n_valid, (long long)N);
+  if (D != 64 && D != 128) return fail(S2_ERR_UNSUPPORTED, "D=%lld: kernels support D in {64, 128}", (long long)D);
+  if (variant == S2_DENSE_CAUSAL) {
+    if (N % s2::kTile) return fail(S2_ERR_UNSUPPORTED, "N=%lld must be a multiple of 128", (long long)N);
+  } else if ((G / 2) % s2::kTile) {
+    return fail(S2_ERR_UNSUPPORTED, "G/2=%lld must be a multiple of 128", (long long)(G / 2));
+  }
+  if (B * N >= (int64_t(1) << 31) || B * H * N >= (int64_t(1) << 31))
+    return fail(S2_ERR_UNSUPPORTED, "B*N and B*H*N must be below 2^31");
+  return S2_OK;
+}
+
+int make_tmap(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t H, int64_t D) {
+  // [B*N, H, D] bf16 viewed as a 3-D tensor (D innermost); box = 64 columns x 1 head x 128 rows.
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(B * N)};
+  cuuint64_t strides[2] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2)};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)s2::kTile};
+  cuuint32_t elem[3] = {1, 1, 1};
+  CUresult r = st->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                          elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(S2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return S2_OK;
+}
+
+int launch_status(int rc, const char* what) {
+  if (rc == 0) return S2_OK;
+  return fail(S2_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString((cudaError_t)rc));
+}
+
+}  // namespace
+
+extern "C" {
+
+int s2attn_version(void) { return 100; }
+
+const char* s2attn_last_error(void) { return g_last_error.c_str(); }
+
+int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
+                 int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* stream) {
+  int rc = validate(B, N, H, D, G, n_valid, variant);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !lse) return fail(S2_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return fail(S2_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  CUtensorMap tq, tk, tv, to;
+  if ((rc = make_tmap(st, &tq, q, B, N, H, D)) || (rc = make_tmap(st, &tk, k, B, N, H, D)) ||
+      (rc = make_tmap(st, &tv, v, B, N, H, D)) || (rc = make_tmap(st, &to, o, B, N, H, D)))
+    return rc;
+  s2::FwdArgs a;
+  a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmO = &to;
+  a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  a.lse = lse;
+  a.status = st->status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_status(s2::launch_fwd(a), "forward");
+}
+
+int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
+               int64_t H, int64_t D, int64_t G, int variant, void* stream) {
+  return s2attn_fwd_v(q, k, v, o, lse, B, N, H, D, G, N, variant, stream);
+}
+
+size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
+  if (B < 1 || N < 1 || H < 1 || D < 1) return 0;
+  const size_t delta = (size_t)B * H * N * sizeof(float);
+  const size_t delta_padded = (delta + 255) / 256 * 256;
+  return delta_padded + (size_t)B * N * H * D * sizeof(float);
+}
+
+int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G,
+                 int64_t n_valid, int variant, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate(B, N, H, D, G, n_valid, variant);
+  if (rc) return rc;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
+    return fail(S2_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(S2_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(S2_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const size_t need = s2attn_bwd_workspace_size(B, N, H, D);
+  if (workspace_bytes < need)
+    return fail(S2_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  if ((rc = make_tmap(st, &tq, q, B, N, H, D)) || (rc = make_tmap(st, &tk, k, B, N, H, D)) ||
+      (rc = make_tmap(st, &tv, v, B, N, H, D)) || (rc = make_tmap(st, &tdo, dout, B, N, H, D)) ||
+      (rc = make_tmap(st, &tdk, dk, B, N, H, D)) || (rc = make_tmap(st, &tdv, dv, B, N, H, D)))
+    return rc;
+  s2::BwdArgs a;
+  a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmdO = &tdo; a.tmdK = &tdk; a.tmdV = &tdv;
+  a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  a.o = o;
+  a.dout = dout;
+  a.lse = lse;
+  const size_t delta = (size_t)B * H * N * sizeof(float);
+  a.delta = static_cast<float*>(workspace);
+  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + (delta + 255) / 256 * 256);
+  a.dq = dq;
+  a.status = st->status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  rc = s2::launch_bwd(a);
+  if (rc == (int)cudaErrorNotSupported) return fail(S2_ERR_UNSUPPORTED, "backward kernel not available");
+  return launch_status(rc, "backward");
+}
+
+int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int variant,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  return s2attn_bwd_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, N, variant, workspace, workspace_bytes,
+                      stream);
+}
+
+int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class, int format,
+                           void* out, void* stream) {
+  // D does not enter the pattern; validate with a supported D.
+  int rc = validate(1, N, 2, 128, G, n_valid, variant);
+  if (rc) return rc;
+  if (head_class != 0 && head_class != 1) return fail(S2_ERR_INVALID_ARG, "head_class must be 0 or 1");
+  if (format != 0 && format != 1) return fail(S2_ERR_INVALID_ARG, "format must be 0 (bits) or 1 (intervals)");
+  if (format == 0 && N > 65536) return fail(S2_ERR_UNSUPPORTED, "bit format supports N <= 65536");
+  if (!out) return fail(S2_ERR_INVALID_ARG, "null output pointer");
+  if (!aligned16(out)) return fail(S2_ERR_INVALID_ARG, "output must be 16-byte aligned");
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  s2::Plan p = s2::make_plan(1, (int)N, 2, 128, (int)G, (int)n_valid, variant);
+  const int cls = (variant == S2_DENSE_CAUSAL) ? 0 : head_class;
+  return launch_status(s2::launch_adjacency(p, cls, format, out, static_cast<cudaStream_t>(stream)), "adjacency");
+}
+
+int s2attn_check_status(void* stream) {
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  int flags = 0;
+  e = cudaMemcpyFromSymbol(&flags, g_s2_status, sizeof(int));
+  if (e != cudaSuccess) return fail(S2_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(e));
+  if (flags) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_s2_status, &zero, sizeof(int));
+    return fail(S2_ERR_TIMEOUT, "a kernel gave up waiting on a barrier (role flags 0x%x)", flags);
+  }
+  return S2_OK;
+}
+
+}  // extern "C"

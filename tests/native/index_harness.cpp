@@ -1,0 +1,49 @@
+// Host replica of the kernels' traversal, built with g++ from the same
+// scheduler header the CUDA kernels include (s2_index.cuh).  Used by
+// tests/test_index_host.py to check the work decomposition and masks on the
+// CPU against the oracle's visibility matrices, exhaustively for small N.
+#include <cstdint>
+#include <cstring>
+
+#include "s2_index.cuh"
+
+extern "C" {
+
+// visited[i*N + j] += 1 for every (query i, key j) pair the kernels compute
+// for a head of class `cls`; cover[i] += 1 for every query row a unit owns.
+// Returns the number of work units decoded (non-idle).
+int s2h_visit(int N, int G, int n_valid, int variant, int cls, uint8_t* visited, int32_t* cover) {
+  s2::Plan p = s2::make_plan(1, N, 2, 128, G, n_valid, variant);
+  int units = 0;
+  for (int L = 0; L < p.ranks * p.B * p.H; ++L) {
+    s2::Unit u;
+    if (!s2::decode_unit(p, L, u)) continue;
+    if (u.h != cls) continue;  // with H = 2, head h has class h (dense: head 0)
+    ++units;
+    for (int x = 0; x < 2; ++x) {
+      if (u.t[x] < 0) continue;
+      const int q0 = s2::tile_orig(p, u, u.t[x]);
+      for (int r = 0; r < s2::kTile; ++r) cover[q0 + r] += 1;
+      for (int k = 0; k <= u.kmax; ++k) {
+        if (!s2::ktile_valid(p, u, k) || !s2::tile_takes(p, u, x, k)) continue;
+        const int k0 = s2::tile_orig(p, u, k);
+        for (int r = 0; r < s2::kTile; ++r) {
+          const int lim = s2::col_limit(p, u, u.t[x], k, r);
+          for (int c = 0; c < lim; ++c) visited[(size_t)(q0 + r) * N + (k0 + c)] += 1;
+        }
+      }
+    }
+  }
+  return units;
+}
+
+// Grid size and per-class unit counts of a launch.
+void s2h_plan(int B, int N, int H, int G, int n_valid, int variant, int32_t* out) {
+  s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);
+  out[0] = p.ranks * p.B * p.H;
+  out[1] = p.nseg[0];
+  out[2] = p.nseg[1];
+  out[3] = p.nunit[0];
+  out[4] = p.nunit[1];
+}
+}

@@ -1,0 +1,138 @@
+"""CPU checks of the kernels' scheduler (s2_index.cuh) and of the C ABI host layer.
+
+The scheduler header is compiled with g++ into a small host harness that walks
+work units, key tiles and column limits exactly as the kernels do; the pairs
+it visits must equal the oracle's explicit matrices A^(0), A^(1) (every pair
+once, nothing else), and every query row must be owned by exactly one unit.
+"""
+from __future__ import annotations
+
+import ctypes
+import re
+import subprocess
+from pathlib import Path
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = Path(__file__).resolve().parent.parent
+CSRC = ROOT / "shifted_sparse_attention_b200" / "csrc"
+HARNESS = Path(__file__).resolve().parent / "native" / "index_harness.cpp"
+
+
+@pytest.fixture(scope="module")
+def harness(tmp_path_factory):
+    out = tmp_path_factory.mktemp("harness") / "libindex_harness.so"
+    subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-I", str(CSRC), str(HARNESS),
+                           "-o", str(out)])
+    L = ctypes.CDLL(str(out))
+    L.s2h_visit.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p]
+    L.s2h_visit.restype = ctypes.c_int
+    L.s2h_plan.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p]
+    return L
+
+
+def _visit(L, N, G, nv, variant, cls):
+    vis = np.zeros((N, N), dtype=np.uint8)
+    cover = np.zeros(N, dtype=np.int32)
+    L.s2h_visit(N, G, nv, variant, cls, vis.ctypes.data, cover.ctypes.data)
+    return vis, cover
+
+
+CASES = [(N, G) for N in (256, 512, 768, 1024, 1536, 2048) for G in (256, 512, 768, 1024) if N % G == 0]
+
+
+@pytest.mark.parametrize("N,G", CASES)
+@pytest.mark.parametrize("variant", [0, 1])
+def test_scheduler_visits_exactly_the_oracle_pairs(harness, N, G, variant):
+    for nv in sorted({N, N - 1, N - 127, N - 128, N - G // 2 - 3, 1, 129, (N * 3) // 5}):
+        if nv < 1:
+            continue
+        for cls in (0, 1):
+            vis, cover = _visit(harness, N, G, nv, variant, cls)
+            A = oracle.adjacency(N, G, nv, variant, cls)
+            assert (cover == 1).all(), (N, G, nv, variant, cls)
+            assert vis.max() <= 1, "a pair was computed twice"
+            np.testing.assert_array_equal(vis.astype(bool), A, err_msg=str((N, G, nv, variant, cls)))
+
+
+@pytest.mark.parametrize("N", [128, 256, 640, 1024])
+def test_scheduler_dense_causal(harness, N):
+    for nv in (N, N - 5, 1):
+        vis, cover = _visit(harness, N, N, nv, 2, 0)
+        assert (cover == 1).all()
+        np.testing.assert_array_equal(vis.astype(bool), oracle.adjacency(N, N, nv, 2, 0))
+
+
+def test_grid_sizes_of_the_workloads(harness):
+    out = np.zeros(5, dtype=np.int32)
+    # long-context workload: 4 unshifted segments of 32 units, 5 strict shifted segments
+    harness.s2h_plan(1, 32768, 32, 8192, 32768, 0, out.ctypes.data)
+    assert out.tolist() == [32 * 5 * 32, 4, 5, 32, 32]
+    harness.s2h_plan(1, 1024, 8, 256, 1024, 0, out.ctypes.data)
+    assert out.tolist() == [8 * 5 * 1, 4, 5, 1, 1]
+
+
+# ---------------------------------------------------------------- C ABI host layer (no GPU needed)
+
+
+@pytest.fixture(scope="module")
+def abi():
+    from shifted_sparse_attention_b200 import build
+    build.build()
+    from shifted_sparse_attention_b200 import binding
+    return binding
+
+
+def test_library_exports_every_declared_symbol(abi):
+    header = (ROOT / "include" / "s2attn.h").read_text()
+    declared = set(re.findall(r"\b(s2attn_\w+)\s*\(", header))
+    assert declared == set(abi.SIGNATURES), declared ^ set(abi.SIGNATURES)
+    nm = subprocess.run(["nm", "-D", "--defined-only", str(abi.LIB_PATH)], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (s2attn_\w+)", nm))
+    assert declared <= exported, declared - exported
+    L = abi.lib()
+    for name in declared:
+        assert hasattr(L, name)
+    assert L.s2attn_version() == 100
+
+
+def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
+    L = abi.lib()
+    fake = 1 << 20  # never dereferenced: validation fails first
+    cases = [
+        (dict(H=3), abi.S2_ERR_SHAPE),           # odd head count
+        (dict(G=255), abi.S2_ERR_SHAPE),         # odd group
+        (dict(N=1000), abi.S2_ERR_SHAPE),        # N not a multiple of G
+        (dict(nv=0), abi.S2_ERR_SHAPE),
+        (dict(nv=1025), abi.S2_ERR_SHAPE),
+        (dict(D=96), abi.S2_ERR_UNSUPPORTED),
+        (dict(G=128), abi.S2_ERR_UNSUPPORTED),   # shift 64 is not a multiple of 128
+        (dict(variant=7), abi.S2_ERR_INVALID_ARG),
+    ]
+    for over, code in cases:
+        a = dict(B=1, N=1024, H=8, D=64, G=256, nv=1024, variant=0)
+        a.update(over)
+        rc = L.s2attn_fwd_v(fake, fake, fake, fake, fake, a["B"], a["N"], a["H"], a["D"], a["G"], a["nv"],
+                            a["variant"], None)
+        assert rc == code, (over, rc, abi.s2attn_last_error())
+        assert abi.s2attn_last_error()
+    rc = L.s2attn_fwd_v(None, fake, fake, fake, fake, 1, 1024, 8, 64, 256, 1024, 0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG
+    rc = L.s2attn_fwd_v(fake + 8, fake, fake, fake, fake, 1, 1024, 8, 64, 256, 1024, 0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # misaligned
+    ws = L.s2attn_bwd_workspace_size(1, 1024, 8, 64)
+    assert ws == 1024 * 8 * 4 + 1024 * 8 * 64 * 4
+    rc = L.s2attn_bwd_v(*([fake] * 9), 1, 1024, 8, 64, 256, 1024, 0, fake, ws - 1, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # workspace too small
+    rc = L.s2attn_debug_adjacency(1024, 256, 1024, 0, 2, 0, fake, None)
+    assert rc == abi.S2_ERR_INVALID_ARG
+
+
+def test_tensor_api_refuses_cpu_tensors(abi):
+    import torch
+    q = torch.zeros(1, 1024, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        abi.forward(q, q, q, 256)
