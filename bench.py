@@ -1,0 +1,428 @@
+"""Benchmark: S²-Attn forward + backward useful TFLOP/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step = one pass of the whole hot path over one batch: s2attn_fwd, then
+the three backward stages (prepare, main, dq finish), on inputs resident in
+HBM.  Default workload: B=1, H=32, N=32768, D=128, G=8192, strict variant,
+bf16 Q/K/V/dO ~ N(0,1) with K doubled on 5% of positions.
+
+Metric: useful causal TFLOP/s = 7·B·H·N·G·D per step (forward 2·B·H·N·G·D,
+backward 2.5x that) / step time; N>1 runs one independent replica per GPU
+(weak scaling, no collective on the data path) and reports the whole-job
+aggregate over the max-over-ranks device time.  Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle (the only reference this
+method has) on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "S²-Attn fwd+bwd useful TFLOP/s at 1 B200 and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="long_n32768_g8192")
+    ap.add_argument("--variant", type=int, default=None, help="0 strict, 1 rolled, 2 dense causal")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"bf16_burst": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
+                "hbm_gbs": d["hbm_gbs"], "source": "measured"}
+    return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def pair_counts(w, variant):
+    """Exact visited (query, key) pairs per head class, closed forms of the grouping."""
+    N, G, nv = w.N, w.G, w.valid
+    tri = lambda L: L * (L + 1) // 2
+    if nv != N:
+        return None
+    s, M = G // 2, N // G
+    if variant == 2:
+        return tri(N), tri(N)
+    c0 = M * tri(G)
+    c1 = c0 if variant == 1 else 2 * tri(s) + (M - 1) * tri(G)
+    return c0, c1
+
+
+# ---------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], swp=parts[8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("swp", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(r["power"] for r in rows)}
+
+
+# ---------------------------------------------------------------------------- CPU oracle leg
+
+
+def oracle_sample(x, w, variant, rows_per_window):
+    """Run the oracle on the last `rows_per_window` query rows of the first
+    full group of every head (fwd + bwd); return (seconds, useful FLOPs of the
+    sample on the metric's formula, threads, description)."""
+    import oracle
+
+    G = w.G
+    r0, r1 = G - rows_per_window, G
+    t0 = time.perf_counter()
+    oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, n_valid=w.n_valid, rows=(r0, r1))
+    dt = time.perf_counter() - t0
+    # exact pairs of the sample (rows r0..r1 of every head), priced at 14·D per pair
+    # (4D forward + 10D backward), then scaled by the metric's formula / exact ratio
+    pc = pair_counts(w, variant)
+    exact_pairs = 0
+    for h in range(w.H):
+        cls = 1 if (h >= w.H // 2 and variant != 2) else 0
+        for i in range(r0, r1):
+            lo = _row_lo(i, G, variant, cls, w.N)
+            exact_pairs += i - lo + 1
+    exact_pairs *= w.B
+    flops_exact = exact_pairs * 14 * w.D
+    ratio = 1.0
+    if pc is not None:
+        ratio = w.formula_flops(passes="fwd+bwd") / (w.B * (w.H // 2) * (pc[0] + pc[1]) * 14 * w.D)
+    desc = ("oracle fwd+bwd on query rows [%d, %d) of all %d heads of the workload's inputs "
+            "(%d visited pairs), priced on the metric's formula" % (r0, r1, w.B * w.H, exact_pairs))
+    return dt, flops_exact * ratio, oracle.num_threads(), desc
+
+
+def _row_lo(i, G, variant, cls, N):
+    s = G // 2
+    if variant == 2:
+        return 0
+    if cls == 0:
+        return (i // G) * G
+    if i < s:
+        return 0
+    return s + ((i - s) // G) * G
+
+
+def run_reference(args, rank, world):
+    import torch  # noqa: F401
+
+    from shifted_sparse_attention_b200 import synthetic
+
+    if rank != 0:
+        return
+    w = synthetic.WORKLOADS[args.workload]
+    variant = w.variants[0] if args.variant is None else args.variant
+    x = synthetic.draw(w.B, w.N, w.H, w.D, seed=w.seed, sharpen_k=w.sharpen_k)
+    rows = 32
+    for _ in range(args.warmup):
+        oracle_sample(x, w, variant, rows)
+    total_t, total_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl, threads, desc = oracle_sample(x, w, variant, rows)
+        total_t += dt
+        total_f += fl
+    value = total_f / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, variant),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, variant):
+    return {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "D": w.D, "G": w.G, "shift": w.G // 2,
+            "group_ratio": w.G / w.N, "n_valid": w.valid,
+            "variant": {0: "strict", 1: "rolled", 2: "dense_causal"}[variant],
+            "l2": "inputs larger than L2 (each of Q/K/V/dO is %d MiB > 126 MB)" % (w.B * w.N * w.H * w.D * 2 >> 20)}
+
+
+def _src_hash(name):
+    return hashlib.sha256((ROOT / "shifted_sparse_attention_b200" / "csrc" / name).read_bytes()).hexdigest()[:16]
+
+
+def _traffic(kernel, src):
+    """Per-launch DRAM bytes from the committed ncu summary, if taken on this exact source."""
+    p = ROOT / "profiles" / "traffic.json"
+    if not p.exists():
+        return None
+    d = json.loads(p.read_text()).get(kernel)
+    if not d or d.get("source_sha256_16") != _src_hash(src):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from shifted_sparse_attention_b200 import binding as s2
+    from shifted_sparse_attention_b200 import synthetic
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synthetic.WORKLOADS[args.workload]
+    variant = w.variants[0] if args.variant is None else args.variant
+    B, N, H, D, G = w.B, w.N, w.H, w.D, w.G
+    x = synthetic.draw(B, N, H, D, seed=w.seed + rank, sharpen_k=w.sharpen_k)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "dout"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q))
+    ws = torch.empty(s2.s2attn_bwd_workspace_size(B, N, H, D), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    nv = w.n_valid
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        s2.forward(q, k, v, G, variant, nv, out=o, lse=lse)
+        if ev is not None:
+            ev[1].record(stream)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE)
+        if ev is not None:
+            ev[2].record(stream)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_MAIN)
+        if ev is not None:
+            ev[3].record(stream)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_FINISH)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    s2.check_status()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    gpu_index = phys[local_rank] if len(phys) > local_rank and phys[local_rank] else str(local_rank)
+    with ClockSampler(gpu_index) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2.check_status()
+    ms = start.elapsed_time(end)
+    per = {name: sum(e[a].elapsed_time(e[b]) for e in evs) / args.steps
+           for name, a, b in (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_main", 2, 3), ("bwd_finish", 3, 4))}
+    clocks = clk.summary()
+
+    # e2e: the same step through the public API from pinned host buffers, copies included
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (q, q, q, q))
+        e_steps = max(1, min(args.steps, 5))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hdq.copy_(grads[0], non_blocking=True)
+            hdk.copy_(grads[1], non_blocking=True)
+            hdv.copy_(grads[2], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e_steps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = a.elapsed_time(b) / e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * w.formula_flops(passes="fwd+bwd") / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes, "ms_per_step": e2e_ms,
+               "steps": e_steps}
+
+    if world > 1:
+        t = torch.tensor([ms] + [per[k] for k in per], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0].item())
+        for i, kname in enumerate(per):
+            per[kname] = float(t[1 + i].item())
+        gathered = [None] * world
+        dist.all_gather_object(gathered, clocks)
+        if rank == 0:
+            meds = [c["sm_mhz"] for c in gathered if c["sm_mhz"] is not None]
+            clocks = {"sm_mhz": statistics.median(meds) if meds else None,
+                      "sm_max_mhz": max((c["sm_max_mhz"] or 0) for c in gathered) or None,
+                      "reasons": sorted(set(r for c in gathered for r in c["reasons"])),
+                      "per_rank_sm_mhz": meds}
+
+    # CPU oracle leg (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, threads, desc = oracle_sample({n: x[n] for n in x}, w, variant, 256)
+        cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    if rank != 0:
+        return
+    pk = peaks()
+    ms_step = ms / args.steps
+    flops_step = w.formula_flops(passes="fwd+bwd")
+    value = world * flops_step / (ms_step * 1e-3) / 1e12
+    pc = pair_counts(w, variant)
+    if pc is not None:
+        pairs = w.B * (w.H // 2) * (pc[0] + pc[1])
+    else:
+        pairs = None
+    # dominant kernel: the longer of the forward and the backward main kernel
+    dom = "bwd_main" if per["bwd_main"] >= per["fwd"] else "fwd"
+    per_pair = {"fwd": 4 * D, "bwd_main": 10 * D}[dom]
+    algo = pairs * per_pair if pairs is not None else w.formula_flops(passes="fwd" if dom == "fwd" else "bwd")
+    achieved = algo / (per[dom] * 1e-3) / 1e12
+    src = {"fwd": "s2_fwd.cu", "bwd_main": "s2_bwd.cu"}[dom]
+    roof = {"bound": "tensor", "kernel": {"fwd": "s2_fwd_kernel", "bwd_main": "s2_bwd_kernel"}[dom],
+            "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+            "frac": achieved / pk["bf16_sustained"],
+            "peak_kind": "bf16 sustained (kernel timed inside a long step loop), %s" % pk["source"],
+            "traffic": _traffic({"fwd": "s2_fwd_kernel", "bwd_main": "s2_bwd_kernel"}[dom], src),
+            "algorithmic_flops_per_launch": algo, "avg_launch_ms": per[dom]}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(_config(w, variant), parallelism="replicas%d" % world if world > 1 else "single"),
+        "pct_of_peak": {"bf16_burst": value / world / pk["bf16_burst"],
+                        "bf16_sustained": value / world / pk["bf16_sustained"],
+                        "nominal_2250": value / world / 2250.0},
+        "kernel_ms": per,
+        "useful_flops_per_step": flops_step,
+        "exact_pair_tflops": (world * pairs * 14 * D / (ms_step * 1e-3) / 1e12) if pairs else None,
+        "clocks": clocks,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

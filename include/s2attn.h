@@ -79,8 +79,9 @@ int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* ls
                  int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
                  void* stream);
 
-/* Bytes of device workspace s2attn_bwd needs: a float32 row statistic
- * Delta_i = dout_i·o_i ([B,H,N]) and a float32 dq accumulator ([B,N,H,D]). */
+/* Bytes of device workspace s2attn_bwd needs: two float32 row statistics
+ * ([B,H,N] each: Delta_i = dout_i·o_i and lse_i·log2(e)) and a float32 dq
+ * accumulator ([B,N,H,D]), each part starting on a 256-byte boundary. */
 size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D);
 
 /* Backward.  Inputs q, k, v, o, dout (bf16), lse (fp32) as produced by the
@@ -97,6 +98,24 @@ int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H,
                  int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace,
                  size_t workspace_bytes, void* stream);
+
+/* The backward is three launches on `stream`; s2attn_bwd_v runs all of them
+ * in order.  Running them one at a time (same arguments, `stages` a bit set)
+ * lets a caller time or overlap them separately:
+ *   S2_BWD_PREPARE  Delta_i = dout_i·o_i, lse_i·log2(e) and a zeroed dq
+ *                   accumulator in the workspace (reads o, dout, lse);
+ *   S2_BWD_MAIN     dk, dv, and the dq accumulator (reads q, k, v, dout and
+ *                   the workspace written by the prepare stage);
+ *   S2_BWD_FINISH   dq = bf16(accumulator / sqrt(D)).
+ * A stage assumes the earlier stages of the same call sequence have run on
+ * the same stream with the same workspace. */
+enum { S2_BWD_PREPARE = 1, S2_BWD_MAIN = 2, S2_BWD_FINISH = 4, S2_BWD_ALL = 7 };
+
+int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
+                        int variant, void* workspace, size_t workspace_bytes, int stages,
+                        void* stream);
 
 /* Debug: the (query, key) pairs the kernels visit for one head class
  * (0: heads [0,H/2), 1: heads [H/2,H); ignored for S2_DENSE_CAUSAL), computed

@@ -27,6 +27,8 @@ SIGNATURES = {
                     _vp, _sz, _vp], _int),
     "s2attn_bwd_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                       _int, _vp, _sz, _vp], _int),
+    "s2attn_bwd_stages_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
+                             _int, _vp, _sz, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
@@ -107,6 +109,16 @@ def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, variant, worksp
                             _ptr(dv), B, N, H, D, G, variant, _ptr(workspace), workspace_bytes, _stream(stream))
 
 
+S2_BWD_PREPARE, S2_BWD_MAIN, S2_BWD_FINISH, S2_BWD_ALL = 1, 2, 4, 7
+
+
+def s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,
+                        workspace_bytes, stages, stream=None) -> int:
+    return lib().s2attn_bwd_stages_v(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                     _ptr(dk), _ptr(dv), B, N, H, D, G, n_valid, variant, _ptr(workspace),
+                                     workspace_bytes, stages, _stream(stream))
+
+
 def s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, out, stream=None) -> int:
     return lib().s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, _ptr(out), _stream(stream))
 
@@ -139,7 +151,7 @@ def forward(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None, 
 
 
 def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int | None = None,
-             grads=None, workspace=None, stream=None):
+             grads=None, workspace=None, stream=None, stages: int = 7):
     """S²-Attn backward; returns (dq, dk, dv) bf16 [B,N,H,D]."""
     B, N, H, D = _shape(q)
     nv = N if n_valid is None else int(n_valid)
@@ -149,8 +161,8 @@ def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int 
     ws_bytes = s2attn_bwd_workspace_size(B, N, H, D)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    _check(s2attn_bwd_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, nv, variant, workspace,
-                        workspace.numel() * workspace.element_size(), stream))
+    _check(s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, nv, variant, workspace,
+                               workspace.numel() * workspace.element_size(), stages, stream))
     return dq, dk, dv
 
 

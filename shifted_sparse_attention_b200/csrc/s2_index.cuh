@@ -40,7 +40,9 @@ struct Plan {
   int B, N, H, D, G, s, n_valid, variant;
   int nseg[2];     // segments per head class
   int nunit[2];    // max work units (pairs of q tiles) per segment, per class
-  int ranks;       // max over classes of nseg * nunit
+  int ranks;       // max over classes of nseg * nunit (forward grid = ranks * B * H)
+  int ntile[2];    // max tiles per segment, per class
+  int kv_ranks;    // max over classes of nseg * ntile (backward grid = kv_ranks * B * H)
   float scale_log2;  // log2(e) / sqrt(D)
 };
 
@@ -156,6 +158,43 @@ S2_HD int col_limit(const Plan& p, const Unit& u, int tq, int k, int r) {
   return lim < kv ? lim : kv;
 }
 
+// ---------------------------------------------------------------- backward units
+// The backward runs one CTA per key tile (128 keys) of a segment and walks the
+// query tiles from the diagonal to the end of the segment.  The unit reuses
+// Unit: t[0] = key tile, t[1] = -1, part[0] = the key tile holds a valid key,
+// kmax = last query tile of the segment.
+
+// Decode a linear backward work index (key tiles with the most query tiles first).
+S2_HD bool decode_kv_unit(const Plan& p, int L, Unit& u) {
+  const int BH = p.B * p.H;
+  const int bh = L % BH, r = L / BH;
+  u.b = bh / p.H;
+  u.h = bh % p.H;
+  u.cls = head_class(p, u.h);
+  const int S = p.nseg[u.cls], NT = p.ntile[u.cls];
+  if (r >= S * NT) return false;
+  const int kt = r / S, seg = r % S;
+  int len;
+  seg_bounds(p, u.cls, seg, u.vbeg, len);
+  u.ntiles = len / kTile;
+  if (kt >= u.ntiles) return false;
+  u.t[0] = kt;
+  u.t[1] = -1;
+  u.part[0] = tile_orig(p, u, kt) < p.n_valid;
+  u.part[1] = false;
+  u.kmax = u.ntiles - 1;
+  return true;
+}
+
+// Queries of query tile qt visible from local key row j of key tile kt:
+// columns [lo, hi).  The same set as col_limit, seen from the key side.
+S2_HD void query_range(const Plan& p, const Unit& u, int kt, int qt, int j, int& lo, int& hi) {
+  lo = (kt == qt) ? j : 0;
+  if (tile_orig(p, u, kt) + j >= p.n_valid) { hi = 0; return; }
+  const int qv = p.n_valid - tile_orig(p, u, qt);
+  hi = qv < kTile ? qv : kTile;
+}
+
 // Host-side plan construction (validated by the caller).
 inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int variant) {
   Plan p{};
@@ -171,9 +210,12 @@ inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int varian
     }
     const int nt = maxlen / kTile;
     p.nunit[c] = (nt + 1) / 2;
+    p.ntile[c] = nt;
   }
   const int r0 = p.nseg[0] * p.nunit[0], r1 = p.nseg[1] * p.nunit[1];
   p.ranks = r0 > r1 ? r0 : r1;
+  const int k0 = p.nseg[0] * p.ntile[0], k1 = p.nseg[1] * p.ntile[1];
+  p.kv_ranks = k0 > k1 ? k0 : k1;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   return p;
 }

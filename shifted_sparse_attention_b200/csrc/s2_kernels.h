@@ -30,7 +30,8 @@ struct BwdArgs {
   const void* o;      // bf16 [B, N, H, D]
   const void* dout;   // bf16 [B, N, H, D]
   const float* lse;   // [B, H, N]
-  float* delta;       // workspace [B, H, N]
+  float* delta;       // workspace [B, H, N]: dout_i·o_i
+  float* lse2;        // workspace [B, H, N]: lse_i·log2(e), +inf on padded rows
   float* dq_acc;      // workspace [B, N, H, D] fp32
   void* dq;           // bf16 [B, N, H, D]
   int* status;
@@ -38,7 +39,8 @@ struct BwdArgs {
 };
 
 int launch_fwd(const FwdArgs& a);
-int launch_bwd(const BwdArgs& a);
+// stages: 1 = prepare (Delta, lse2, zero accumulator), 2 = main, 4 = dq convert.
+int launch_bwd(const BwdArgs& a, int stages);
 int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
 
 }  // namespace s2

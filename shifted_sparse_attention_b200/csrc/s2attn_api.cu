@@ -56,6 +56,10 @@ int device_state(DeviceState** out) {
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(S2_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  // Make the device's primary context current on this thread (callers such as
+  // autograd worker threads may not have touched the runtime yet).
+  e = cudaSetDevice(dev);
+  if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaSetDevice: %s", cudaGetErrorString(e));
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& st = g_dev[dev];
   if (!st.ready) {
@@ -164,16 +168,22 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return s2attn_fwd_v(q, k, v, o, lse, B, N, H, D, G, N, variant, stream);
 }
 
-size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
-  if (B < 1 || N < 1 || H < 1 || D < 1) return 0;
-  const size_t delta = (size_t)B * H * N * sizeof(float);
-  const size_t delta_padded = (delta + 255) / 256 * 256;
-  return delta_padded + (size_t)B * N * H * D * sizeof(float);
+// Workspace = [Delta: B*H*N f32][lse*log2(e): B*H*N f32][dq accumulator: B*N*H*D f32],
+// each part starting on a 256-byte boundary.
+static size_t stat_bytes(int64_t B, int64_t N, int64_t H) {
+  return ((size_t)B * H * N * sizeof(float) + 255) / 256 * 256;
 }
 
-int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
-                 void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G,
-                 int64_t n_valid, int variant, void* workspace, size_t workspace_bytes, void* stream) {
+size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
+  if (B < 1 || N < 1 || H < 1 || D < 1) return 0;
+  return 2 * stat_bytes(B, N, H) + (size_t)B * N * H * D * sizeof(float);
+}
+
+int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D,
+                        int64_t G, int64_t n_valid, int variant, void* workspace, size_t workspace_bytes,
+                        int stages, void* stream) {
+  if (stages < 1 || stages > S2_BWD_ALL) return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7");
   int rc = validate(B, N, H, D, G, n_valid, variant);
   if (rc) return rc;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
@@ -199,15 +209,21 @@ int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, con
   a.o = o;
   a.dout = dout;
   a.lse = lse;
-  const size_t delta = (size_t)B * H * N * sizeof(float);
+  const size_t sb = stat_bytes(B, N, H);
   a.delta = static_cast<float*>(workspace);
-  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + (delta + 255) / 256 * 256);
+  a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
+  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * sb);
   a.dq = dq;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
-  rc = s2::launch_bwd(a);
-  if (rc == (int)cudaErrorNotSupported) return fail(S2_ERR_UNSUPPORTED, "backward kernel not available");
-  return launch_status(rc, "backward");
+  return launch_status(s2::launch_bwd(a, stages), "backward");
+}
+
+int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G,
+                 int64_t n_valid, int variant, void* workspace, size_t workspace_bytes, void* stream) {
+  return s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,
+                             workspace_bytes, S2_BWD_ALL, stream);
 }
 
 int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,

@@ -37,6 +37,33 @@ int s2h_visit(int N, int G, int n_valid, int variant, int cls, uint8_t* visited,
   return units;
 }
 
+// Same as s2h_visit for the backward's key-tile units: visited[i*N + j] += 1
+// for every pair the backward computes; cover[j] += 1 per key row owned.
+int s2h_visit_bwd(int N, int G, int n_valid, int variant, int cls, uint8_t* visited, int32_t* cover) {
+  s2::Plan p = s2::make_plan(1, N, 2, 128, G, n_valid, variant);
+  int units = 0;
+  for (int L = 0; L < p.kv_ranks * p.B * p.H; ++L) {
+    s2::Unit u;
+    if (!s2::decode_kv_unit(p, L, u)) continue;
+    if (u.h != cls) continue;
+    ++units;
+    const int kt = u.t[0];
+    const int k0 = s2::tile_orig(p, u, kt);
+    for (int j = 0; j < s2::kTile; ++j) cover[k0 + j] += 1;
+    if (!u.part[0]) continue;
+    for (int qt = kt; qt <= u.kmax; ++qt) {
+      if (!s2::ktile_valid(p, u, qt)) continue;
+      const int q0 = s2::tile_orig(p, u, qt);
+      for (int j = 0; j < s2::kTile; ++j) {
+        int lo, hi;
+        s2::query_range(p, u, kt, qt, j, lo, hi);
+        for (int i = lo; i < hi; ++i) visited[(size_t)(q0 + i) * N + (k0 + j)] += 1;
+      }
+    }
+  }
+  return units;
+}
+
 // Grid size and per-class unit counts of a launch.
 void s2h_plan(int B, int N, int H, int G, int n_valid, int variant, int32_t* out) {
   s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);

@@ -1,0 +1,85 @@
+"""Backward parity of libs2attn.so against the float64 oracle (needs a B200)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from shifted_sparse_attention_b200 import binding as s2
+from shifted_sparse_attention_b200 import synthetic
+from tests.tolerance import check_grad, check_o, to_np
+
+pytestmark = pytest.mark.gpu
+
+STRICT, ROLLED, DENSE = 0, 1, 2
+
+
+def _run(x, G, variant, nv=None):
+    dev = {n: t.cuda() for n, t in x.items()}
+    o, lse = s2.forward(dev["q"], dev["k"], dev["v"], G, variant, nv)
+    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, G, variant, nv)
+    s2.check_status()
+    return o.cpu(), dq.cpu(), dk.cpu(), dv.cpu()
+
+
+CASES = [
+    # (B, N, H, D, G, variant, n_valid)
+    (1, 1024, 8, 64, 256, STRICT, None),      # small workload, whole
+    (1, 1024, 8, 64, 256, ROLLED, None),
+    (1, 1024, 4, 64, 512, STRICT, 1000),
+    (2, 2048, 4, 128, 512, STRICT, None),
+    (2, 2048, 4, 128, 512, ROLLED, None),
+    (2, 2048, 4, 128, 512, STRICT, 1900),
+    (2, 2048, 4, 128, 512, ROLLED, 1283),
+    (1, 2048, 4, 128, 2048, DENSE, None),
+    (1, 1536, 4, 128, 768, DENSE, 1409),
+    (1, 1536, 2, 128, 768, STRICT, 129),
+    (1, 4096, 2, 128, 1024, ROLLED, 3000),
+]
+
+
+@pytest.mark.parametrize("B,N,H,D,G,variant,nv", CASES)
+def test_backward_matches_oracle(B, N, H, D, G, variant, nv):
+    x = synthetic.draw(B, N, H, D, seed=2000 + N + G + variant)
+    o, dq, dk, dv = _run(x, G, variant, nv)
+    ref = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, n_valid=nv)
+    where = str((B, N, H, D, G, variant, nv))
+    check_o(o, ref["o"], where)
+    n = N if nv is None else nv
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check_grad(name, to_np(g)[:, :n], ref[name][:, :n], where)
+        if nv is not None:
+            assert (to_np(g)[:, nv:] == 0).all(), (name, where)
+
+
+def test_backward_sharpened_keys_small():
+    x = synthetic.draw(1, 2048, 4, 128, seed=5, sharpen_k=True)
+    o, dq, dk, dv = _run(x, 1024, STRICT)
+    ref = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=1024, variant=STRICT)
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        check_grad(name, g, ref[name])
+
+
+def test_backward_padding_values_do_not_matter():
+    B, N, H, D, G, nv = 1, 2048, 4, 128, 512, 1700
+    x = synthetic.draw(B, N, H, D, seed=8)
+    y = {n: t.clone() for n, t in x.items()}
+    for n in y:
+        y[n][:, nv:] = (torch.randn_like(y[n][:, nv:].float()) * 9).to(torch.bfloat16)
+    for variant in (STRICT, ROLLED):
+        a = _run(x, G, variant, nv)
+        b = _run(y, G, variant, nv)
+        for ta, tb in zip(a, b):
+            assert torch.equal(ta[:, :nv], tb[:, :nv])
+            assert (ta[:, nv:] == 0).all() and (tb[:, nv:] == 0).all()
+
+
+def test_autograd_wrapper_runs_library_backward():
+    x = synthetic.draw(1, 1024, 4, 128, seed=9)
+    q, k, v = (x[n].cuda().requires_grad_(True) for n in ("q", "k", "v"))
+    o = s2.s2_attention(q, k, v, 512, STRICT)
+    o.backward(x["dout"].cuda())
+    ref = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=512, variant=STRICT)
+    for name, t in (("dq", q), ("dk", k), ("dv", v)):
+        check_grad(name, t.grad, ref[name])

@@ -30,14 +30,17 @@ def harness(tmp_path_factory):
     L = ctypes.CDLL(str(out))
     L.s2h_visit.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p]
     L.s2h_visit.restype = ctypes.c_int
+    L.s2h_visit_bwd.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p]
+    L.s2h_visit_bwd.restype = ctypes.c_int
     L.s2h_plan.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p]
     return L
 
 
-def _visit(L, N, G, nv, variant, cls):
+def _visit(L, N, G, nv, variant, cls, backward=False):
     vis = np.zeros((N, N), dtype=np.uint8)
     cover = np.zeros(N, dtype=np.int32)
-    L.s2h_visit(N, G, nv, variant, cls, vis.ctypes.data, cover.ctypes.data)
+    fn = L.s2h_visit_bwd if backward else L.s2h_visit
+    fn(N, G, nv, variant, cls, vis.ctypes.data, cover.ctypes.data)
     return vis, cover
 
 
@@ -51,19 +54,22 @@ def test_scheduler_visits_exactly_the_oracle_pairs(harness, N, G, variant):
         if nv < 1:
             continue
         for cls in (0, 1):
-            vis, cover = _visit(harness, N, G, nv, variant, cls)
             A = oracle.adjacency(N, G, nv, variant, cls)
-            assert (cover == 1).all(), (N, G, nv, variant, cls)
-            assert vis.max() <= 1, "a pair was computed twice"
-            np.testing.assert_array_equal(vis.astype(bool), A, err_msg=str((N, G, nv, variant, cls)))
+            for backward in (False, True):
+                vis, cover = _visit(harness, N, G, nv, variant, cls, backward)
+                where = str((N, G, nv, variant, cls, "bwd" if backward else "fwd"))
+                assert (cover == 1).all(), where
+                assert vis.max() <= 1, "a pair was computed twice " + where
+                np.testing.assert_array_equal(vis.astype(bool), A, err_msg=where)
 
 
 @pytest.mark.parametrize("N", [128, 256, 640, 1024])
 def test_scheduler_dense_causal(harness, N):
     for nv in (N, N - 5, 1):
-        vis, cover = _visit(harness, N, N, nv, 2, 0)
-        assert (cover == 1).all()
-        np.testing.assert_array_equal(vis.astype(bool), oracle.adjacency(N, N, nv, 2, 0))
+        for backward in (False, True):
+            vis, cover = _visit(harness, N, N, nv, 2, 0, backward)
+            assert (cover == 1).all()
+            np.testing.assert_array_equal(vis.astype(bool), oracle.adjacency(N, N, nv, 2, 0))
 
 
 def test_grid_sizes_of_the_workloads(harness):
@@ -124,7 +130,7 @@ def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
     rc = L.s2attn_fwd_v(fake + 8, fake, fake, fake, fake, 1, 1024, 8, 64, 256, 1024, 0, None)
     assert rc == abi.S2_ERR_INVALID_ARG  # misaligned
     ws = L.s2attn_bwd_workspace_size(1, 1024, 8, 64)
-    assert ws == 1024 * 8 * 4 + 1024 * 8 * 64 * 4
+    assert ws == 2 * 1024 * 8 * 4 + 1024 * 8 * 64 * 4
     rc = L.s2attn_bwd_v(*([fake] * 9), 1, 1024, 8, 64, 256, 1024, 0, fake, ws - 1, None)
     assert rc == abi.S2_ERR_INVALID_ARG  # workspace too small
     rc = L.s2attn_debug_adjacency(1024, 256, 1024, 0, 2, 0, fake, None)
