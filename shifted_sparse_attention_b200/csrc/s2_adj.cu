@@ -66,7 +66,7 @@ int launch_adjacency(const Plan& p0, int head_class, int format, void* out, cuda
   // rows that no tile covers cannot exist, but start from a defined state
   if (format == 1)
     s2_fill_kernel<<<64, 256, 0, stream>>>(static_cast<int*>(out), (size_t)p.N * 4, -1);
-  const int grid = p.ranks * 2;
+  const int grid = grid_fwd(p);
   s2_adjacency_kernel<<<grid, 256, 0, stream>>>(p, head_class, format, static_cast<uint32_t*>(out),
                                                 static_cast<int*>(out));
   return (int)cudaGetLastError();

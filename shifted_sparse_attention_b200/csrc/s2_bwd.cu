@@ -428,6 +428,343 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ split backward kernel (D = 128)
+// Same CTA decomposition (one 128-key tile, query tiles from the diagonal to
+// the segment end), but every query tile is processed as two 64-query halves,
+// half x by warpgroup x, so that one half's elementwise work runs while the
+// tensor core works on the other half:
+//   S^T_x  = K Q_x^T          (M 128 keys, N 64 queries)   TMEM [64x, 64x+64)
+//   dP^T_x = V dO_x^T                                        TMEM [128+64x, ...)
+//   P^T_x (bf16, into the dP^T_x columns), dS^T_x (bf16, shared memory)
+//   dV += P^T_x dO_x (A from TMEM),  dK += dS^T_x Q_x
+//   dQ^T_x = K^T dS^T_x       (M = D = 128, N 64 queries) -> the S^T_x columns
+// dQ^T puts d on the TMEM lanes, so each warp's float32 atomic adds into the
+// dq accumulator cover 128 contiguous bytes of one query row.
+namespace bwds {
+
+constexpr int D = 128;
+constexpr int kThreads = 320;
+constexpr int kStages = 2;
+constexpr int kChunkBytes = kTile * 64 * 2;
+
+enum Bar {
+  KV_FULL = 0,
+  QD_FULL = 1,    // + stage (2)
+  QD_EMPTY = 3,   // + stage (2)
+  SP_FULL = 5,    // + half (2)
+  DS_READY = 7,   // + half (2)
+  DQ_FULL = 9,    // + half (2)
+  DQ_FREE = 11,   // + half (2)
+  ACC_DONE = 13,
+  NUM_BARS = 14
+};
+
+struct Layout {
+  static constexpr int kTileBytes = kTile * D * 2;       // 32 KB
+  static constexpr int kHalfBytes = kTile * 64 * 2;      // 16 KB: dS^T of one half
+  static constexpr int kStatBytes = 2 * kTile * 4;       // lse2[128], delta[128]
+  static constexpr int kK = 0;
+  static constexpr int kV = kTileBytes;
+  static constexpr int kQ = 2 * kTileBytes;
+  static constexpr int kdO = kQ + kStages * kTileBytes;
+  static constexpr int kdS = kdO + kStages * kTileBytes;
+  static constexpr int kStat = kdS + 2 * kHalfBytes;
+  static constexpr int kBars = kStat + kStages * kStatBytes;
+  static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
+};
+
+}  // namespace bwds
+
+__global__ void __launch_bounds__(bwds::kThreads, 1)
+    s2_bwd_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                        const Plan p, const float* __restrict__ delta, const float* __restrict__ lse2,
+                        float* __restrict__ dq_acc, int* __restrict__ status) {
+  using namespace bwds;
+  using L = bwds::Layout;
+  constexpr int kChunks = D / 64;
+
+  Unit u;
+  if (!decode_kv_unit(p, blockIdx.x, u)) return;
+  extern __shared__ __align__(1024) uint8_t smem_split[];
+  // The layout needs a 1024-byte aligned base (128-byte swizzle atoms); the
+  // dynamic window starts aligned in practice.  If it ever does not, report
+  // and leave instead of computing on misaligned tiles.
+  if (smem_u32(smem_split) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(status, 256);
+    return;
+  }
+  const int kt = u.t[0];
+  const int k0 = tile_orig(p, u, kt);
+  const bool kvalid = u.part[0];
+
+  uint8_t* smem = smem_split;
+  const uint32_t sb = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const uint32_t sK = sb + L::kK, sV = sb + L::kV;
+  auto sQ = [&](int st) { return sb + L::kQ + st * L::kTileBytes; };
+  auto sdO = [&](int st) { return sb + L::kdO + st * L::kTileBytes; };
+  auto sdS = [&](int x) { return sb + L::kdS + x * L::kHalfBytes; };
+  auto sStat = [&](int st) { return sb + L::kStat + st * L::kStatBytes; };
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    mbar_init(bar(KV_FULL), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(QD_FULL + i), 1);
+      mbar_init(bar(QD_EMPTY + i), 1);
+      mbar_init(bar(SP_FULL + i), 1);
+      mbar_init(bar(DS_READY + i), 128);
+      mbar_init(bar(DQ_FULL + i), 1);
+      mbar_init(bar(DQ_FREE + i), 128);
+    }
+    mbar_init(bar(ACC_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto tS = [&](int x) { return tmem + 64 * x; };
+  auto tDP = [&](int x) { return tmem + 128 + 64 * x; };
+  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+  const int row_base = u.b * p.N;
+  const size_t stat_base = ((size_t)u.b * p.H + u.h) * p.N;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && kvalid) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmdO);
+      mbar_arrive_expect_tx(bar(KV_FULL), 2 * L::kTileBytes);
+      for (int c = 0; c < kChunks; ++c) {
+        tma_load_3d(sK + c * kChunkBytes, &tmK, c * 64, u.h, row_base + k0, bar(KV_FULL));
+        tma_load_3d(sV + c * kChunkBytes, &tmV, c * 64, u.h, row_base + k0, bar(KV_FULL));
+      }
+      int n = 0;
+      bool ok = true;
+      for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
+        const int st = n % kStages;
+        if (n >= kStages) ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(QD_FULL + st), 2 * L::kTileBytes + L::kStatBytes);
+        const int q0 = tile_orig(p, u, qt);
+        for (int c = 0; c < kChunks; ++c) {
+          tma_load_3d(sQ(st) + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
+          tma_load_3d(sdO(st) + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
+        }
+        bulk_load(sStat(st), lse2 + stat_base + q0, kTile * 4, bar(QD_FULL + st));
+        bulk_load(sStat(st) + kTile * 4, delta + stat_base + q0, kTile * 4, bar(QD_FULL + st));
+        ++n;
+      }
+      for (int d = (n > kStages ? n - kStages : 0); d < n; ++d)
+        s2_wait(bar(QD_FULL + d % kStages), (d / kStages) & 1, abort_flag, status, 8);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && kvalid) {
+      constexpr uint32_t id_sp = umma_idesc_bf16(128, 64, 0, 0);   // S^T_x, dP^T_x
+      constexpr uint32_t id_acc = umma_idesc_bf16(128, D, 0, 1);   // dV (A in TMEM), dK
+      constexpr uint32_t id_dq = umma_idesc_bf16(128, 64, 1, 1);   // dQ^T_x = K^T dS^T_x
+      bool ok = s2_wait(bar(KV_FULL), 0, abort_flag, status, 16);
+      tc_fence_after();
+      int n = 0;
+      for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
+        const int st = n % kStages;
+        ok = s2_wait(bar(QD_FULL + st), (n / kStages) & 1, abort_flag, status, 16);
+        if (!ok) break;
+        tc_fence_after();
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (n > 0) {  // dQ^T_x(n-1) read out of the S columns, P^T_x(n-1) consumed
+            ok = s2_wait(bar(DQ_FREE + x), (n - 1) & 1, abort_flag, status, 16);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          const uint32_t qrow = x * 64 * 128;  // first query row of the half inside a 64-column chunk
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
+            umma_ss(tS(x), umma_desc_sw128(sK + off, 16, 1024), umma_desc_sw128(sQ(st) + off + qrow, 16, 1024),
+                    id_sp, kk > 0);
+          }
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
+            umma_ss(tDP(x), umma_desc_sw128(sV + off, 16, 1024), umma_desc_sw128(sdO(st) + off + qrow, 16, 1024),
+                    id_sp, kk > 0);
+          }
+          umma_commit(bar(SP_FULL + x));
+        }
+        for (int x = 0; x < 2 && ok; ++x) {
+          ok = s2_wait(bar(DS_READY + x), n & 1, abort_flag, status, 16);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t qrow = x * 64 * 128;
+          const bool first = (n == 0 && x == 0);
+          // dV += P^T_x dO_x : K = 64 queries of the half
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ts(tdV, tDP(x) + kk * 8, umma_desc_sw128(sdO(st) + qrow + kk * 2048, kChunkBytes, 1024), id_acc,
+                    (!first || kk > 0) ? 1u : 0u);
+          // dK += dS^T_x Q_x
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(tdK, umma_desc_sw128(sdS(x) + kk * 32, 16, 1024),
+                    umma_desc_sw128(sQ(st) + qrow + kk * 2048, kChunkBytes, 1024), id_acc,
+                    (!first || kk > 0) ? 1u : 0u);
+          // dQ^T_x = K^T dS^T_x : M = D, K = 128 keys
+          for (int kk = 0; kk < kTile / 16; ++kk)
+            umma_ss(tS(x), umma_desc_sw128(sK + kk * 2048, kChunkBytes, 1024),
+                    umma_desc_sw128(sdS(x) + kk * 2048, kChunkBytes, 1024), id_dq, kk > 0 ? 1u : 0u);
+          umma_commit(bar(DQ_FULL + x));
+        }
+        if (!ok) break;
+        umma_commit(bar(QD_EMPTY + st));
+        ++n;
+      }
+      umma_commit(bar(ACC_DONE));
+      s2_wait(bar(ACC_DONE), 0, abort_flag, status, 16);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ elementwise warpgroups
+    const int x = warp / 4;                 // query half [64x, 64x + 64)
+    const int j = (warp % 4) * 32 + lane;   // key row == TMEM lane (also d for dQ^T)
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    bool ok = true;
+    int n = 0;
+    if (kvalid) {
+      for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
+        const int st = n % kStages;
+        const int q0 = tile_orig(p, u, qt);
+        int lo, hi;
+        query_range(p, u, kt, qt, j, lo, hi);
+        // the stage's lse2 / Delta rows come with its Q/dO tiles
+        ok = s2_wait(bar(QD_FULL + st), (n / kStages) & 1, abort_flag, status, 32);
+        if (!ok) break;
+        ok = s2_wait(bar(SP_FULL + x), n & 1, abort_flag, status, 32);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int col0 = 64 * x + 32 * c;  // first query (tile-local) of this chunk
+          uint32_t sv[32], dp[32];
+          tmem_ld32(tS(x) + lane_off + 32 * c, sv);
+          tmem_ld32(tDP(x) + lane_off + 32 * c, dp);
+          tmem_wait_ld();
+          const float* lsv = reinterpret_cast<const float*>(smem + L::kStat + st * L::kStatBytes) + col0;
+          const float* dlv = lsv + kTile;
+          uint32_t pp[16], dsp[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            float pr[2], ds[2];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int col = col0 + i + t;
+              const bool vis = (col >= lo) && (col < hi);
+              const float e = ex2(fmaf(__uint_as_float(sv[i + t]), p.scale_log2, -lsv[i + t]));
+              pr[t] = vis ? e : 0.f;
+              ds[t] = pr[t] * (__uint_as_float(dp[i + t]) - dlv[i + t]);
+            }
+            pp[i / 2] = pack_bf16(pr[0], pr[1]);
+            dsp[i / 2] = pack_bf16(ds[0], ds[1]);
+          }
+          tmem_st16(tDP(x) + lane_off + 16 * c, pp);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int piece = 4 * c + q;
+            st_shared_v4(sdS(x) + j * 128 + ((piece ^ (j & 7)) << 4), dsp[4 * q], dsp[4 * q + 1], dsp[4 * q + 2],
+                         dsp[4 * q + 3]);
+          }
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(DS_READY + x));
+        // dQ^T_x: lane = d, columns = the half's 64 queries
+        ok = s2_wait(bar(DQ_FULL + x), n & 1, abort_flag, status, 32);
+        if (!ok) break;
+        tc_fence_after();
+        const int qfirst = q0 + 64 * x;
+        const int nq = p.n_valid - qfirst;  // valid queries of the half (may be <= 0 or > 64)
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t dq[32];
+          tmem_ld32(tS(x) + lane_off + 32 * c2, dq);
+          tmem_wait_ld();
+          float* dst = dq_acc + ((size_t)(row_base + qfirst + 32 * c2) * p.H + u.h) * D + j;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c2 + i < nq) atomicAdd(dst + (size_t)i * p.H * D, __uint_as_float(dq[i]));
+        }
+        tc_fence_before();
+        mbar_arrive(bar(DQ_FREE + x));
+        ++n;
+      }
+    }
+    // ---------------------------------------------------------- epilogue: dK, dV
+    bool have = kvalid && ok && n > 0;
+    if (have) {
+      have = s2_wait(bar(ACC_DONE), 0, abort_flag, status, 32);
+      tc_fence_after();
+    }
+    const bool key_valid = have && (k0 + j < p.n_valid);
+    const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t tsrc = which == 0 ? tdV : tdK;
+      const float mul = which == 0 ? 1.f : scale;
+      const uint32_t stage = sQ(which);
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int d0 = x * 64 + 32 * c2;
+        uint32_t v[32];
+        if (have) {
+          tmem_ld32(tsrc + lane_off + d0, v);
+          tmem_wait_ld();
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int col = d0 + 8 * q;
+          const int chunk = col / 64, piece = (col % 64) / 8;
+          uint32_t w[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float a = key_valid ? __uint_as_float(v[8 * q + 2 * t]) * mul : 0.f;
+            const float b = key_valid ? __uint_as_float(v[8 * q + 2 * t + 1]) * mul : 0.f;
+            w[t] = pack_bf16(a, b);
+          }
+          st_shared_v4(stage + chunk * kChunkBytes + j * 128 + ((piece ^ (j & 7)) << 4), w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(2, 256);
+    if (threadIdx.x == 0) {
+      for (int c = 0; c < kChunks; ++c) {
+        tma_store_3d(&tmdV, sQ(0) + c * kChunkBytes, c * 64, u.h, row_base + k0);
+        tma_store_3d(&tmdK, sQ(1) + c * kChunkBytes, c * 64, u.h, row_base + k0);
+      }
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 template <int D>
 int launch_bwd_impl(const BwdArgs& a, int stages) {
   using L = bwd::Layout<D>;
@@ -444,11 +781,19 @@ int launch_bwd_impl(const BwdArgs& a, int stages) {
     if (e != cudaSuccess) return (int)e;
   }
   if (stages & 2) {  // main: dK, dV and the dq accumulator
-    e = cudaFuncSetAttribute(s2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-    if (e != cudaSuccess) return (int)e;
-    const int grid = p.kv_ranks * p.B * p.H;
-    s2_bwd_kernel<D><<<grid, bwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK,
-                                                                   *a.tmdV, p, a.delta, a.lse2, a.dq_acc, a.status);
+    const int grid = grid_bwd(p);
+    if (D == 128) {
+      static_assert(bwds::Layout::kBytes <= 232448, "shared memory budget");
+      e = cudaFuncSetAttribute(s2_bwd_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwds::Layout::kBytes);
+      if (e != cudaSuccess) return (int)e;
+      s2_bwd_split_kernel<<<grid, bwds::kThreads, bwds::Layout::kBytes, a.stream>>>(
+          *a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK, *a.tmdV, p, a.delta, a.lse2, a.dq_acc, a.status);
+    } else {
+      e = cudaFuncSetAttribute(s2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+      if (e != cudaSuccess) return (int)e;
+      s2_bwd_kernel<D><<<grid, bwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK,
+                                                                     *a.tmdV, p, a.delta, a.lse2, a.dq_acc, a.status);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;
   }

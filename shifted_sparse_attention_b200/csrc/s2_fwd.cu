@@ -383,7 +383,7 @@ int launch_fwd_impl(const FwdArgs& a) {
   static_assert(L::kAlloc <= 232448, "shared memory budget");
   cudaError_t e = cudaFuncSetAttribute(s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return (int)e;
-  const int grid = a.plan.ranks * a.plan.B * a.plan.H;
+  const int grid = grid_fwd(a.plan);
   s2_fwd_kernel<D><<<grid, fwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmO, a.plan,
                                                                  a.lse, a.status);
   return (int)cudaGetLastError();

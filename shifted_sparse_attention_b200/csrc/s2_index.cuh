@@ -43,8 +43,23 @@ struct Plan {
   int ranks;       // max over classes of nseg * nunit (forward grid = ranks * B * H)
   int ntile[2];    // max tiles per segment, per class
   int kv_ranks;    // max over classes of nseg * ntile (backward grid = kv_ranks * B * H)
+  int hg_fwd, hg_bwd;  // heads interleaved per group of consecutive CTAs (L2 locality)
   float scale_log2;  // log2(e) / sqrt(D)
 };
+
+// Linear CTA index -> (flattened head bh, per-head slot r).  CTAs are issued
+// in groups of `hg` heads; inside a group the slot r is the slow index, so the
+// CTAs resident at one time work on few heads and their K/V (forward) or
+// Q/dO and dq rows (backward) stay in L2, while r still runs longest-first.
+S2_HD bool split_index(const Plan& p, int L, int R, int hg, int& bh, int& r) {
+  const int BH = p.B * p.H;
+  const int grp = L / (hg * R), within = L % (hg * R);
+  r = within / hg;
+  bh = grp * hg + within % hg;
+  return bh < BH;
+}
+
+S2_HD int groups_of(int n, int hg) { return (n + hg - 1) / hg; }
 
 S2_HD int head_class(const Plan& p, int h) {
   return (p.variant == kDenseCausal) ? 0 : (h >= p.H / 2 ? 1 : 0);
@@ -113,8 +128,8 @@ S2_HD int tile_orig(const Plan& p, const Unit& u, int t) {
 
 // Decode a linear work index (longest work first).  Returns false for idle indices.
 S2_HD bool decode_unit(const Plan& p, int L, Unit& u) {
-  const int BH = p.B * p.H;
-  const int bh = L % BH, r = L / BH;
+  int bh, r;
+  if (!split_index(p, L, p.ranks, p.hg_fwd, bh, r)) return false;
   u.b = bh / p.H;
   u.h = bh % p.H;
   u.cls = head_class(p, u.h);
@@ -166,8 +181,8 @@ S2_HD int col_limit(const Plan& p, const Unit& u, int tq, int k, int r) {
 
 // Decode a linear backward work index (key tiles with the most query tiles first).
 S2_HD bool decode_kv_unit(const Plan& p, int L, Unit& u) {
-  const int BH = p.B * p.H;
-  const int bh = L % BH, r = L / BH;
+  int bh, r;
+  if (!split_index(p, L, p.kv_ranks, p.hg_bwd, bh, r)) return false;
   u.b = bh / p.H;
   u.h = bh % p.H;
   u.cls = head_class(p, u.h);
@@ -195,6 +210,10 @@ S2_HD void query_range(const Plan& p, const Unit& u, int kt, int qt, int j, int&
   hi = qv < kTile ? qv : kTile;
 }
 
+// Grid sizes of the forward and backward launches.
+S2_HD int grid_fwd(const Plan& p) { return groups_of(p.B * p.H, p.hg_fwd) * p.hg_fwd * p.ranks; }
+S2_HD int grid_bwd(const Plan& p) { return groups_of(p.B * p.H, p.hg_bwd) * p.hg_bwd * p.kv_ranks; }
+
 // Host-side plan construction (validated by the caller).
 inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int variant) {
   Plan p{};
@@ -216,6 +235,8 @@ inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int varian
   p.ranks = r0 > r1 ? r0 : r1;
   const int k0 = p.nseg[0] * p.ntile[0], k1 = p.nseg[1] * p.ntile[1];
   p.kv_ranks = k0 > k1 ? k0 : k1;
+  p.hg_fwd = 2;
+  p.hg_bwd = 1;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
   return p;
 }

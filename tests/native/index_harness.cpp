@@ -15,7 +15,7 @@ extern "C" {
 int s2h_visit(int N, int G, int n_valid, int variant, int cls, uint8_t* visited, int32_t* cover) {
   s2::Plan p = s2::make_plan(1, N, 2, 128, G, n_valid, variant);
   int units = 0;
-  for (int L = 0; L < p.ranks * p.B * p.H; ++L) {
+  for (int L = 0; L < s2::grid_fwd(p); ++L) {
     s2::Unit u;
     if (!s2::decode_unit(p, L, u)) continue;
     if (u.h != cls) continue;  // with H = 2, head h has class h (dense: head 0)
@@ -42,7 +42,7 @@ int s2h_visit(int N, int G, int n_valid, int variant, int cls, uint8_t* visited,
 int s2h_visit_bwd(int N, int G, int n_valid, int variant, int cls, uint8_t* visited, int32_t* cover) {
   s2::Plan p = s2::make_plan(1, N, 2, 128, G, n_valid, variant);
   int units = 0;
-  for (int L = 0; L < p.kv_ranks * p.B * p.H; ++L) {
+  for (int L = 0; L < s2::grid_bwd(p); ++L) {
     s2::Unit u;
     if (!s2::decode_kv_unit(p, L, u)) continue;
     if (u.h != cls) continue;
@@ -67,7 +67,7 @@ int s2h_visit_bwd(int N, int G, int n_valid, int variant, int cls, uint8_t* visi
 // Grid size and per-class unit counts of a launch.
 void s2h_plan(int B, int N, int H, int G, int n_valid, int variant, int32_t* out) {
   s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);
-  out[0] = p.ranks * p.B * p.H;
+  out[0] = s2::grid_fwd(p);
   out[1] = p.nseg[0];
   out[2] = p.nseg[1];
   out[3] = p.nunit[0];
