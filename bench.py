@@ -38,7 +38,7 @@ UNIT = "TFLOP/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="long_n32768_g8192")
@@ -185,7 +185,7 @@ def run_reference(args, rank, world):
     w = synthetic.WORKLOADS[args.workload]
     variant = w.variants[0] if args.variant is None else args.variant
     x = synthetic.draw(w.B, w.N, w.H, w.D, seed=w.seed, sharpen_k=w.sharpen_k)
-    rows = 32
+    rows = 16  # a ~1-2 s sample per step on a 16-core host
     for _ in range(args.warmup):
         oracle_sample(x, w, variant, rows)
     total_t, total_f = 0.0, 0.0
@@ -280,6 +280,7 @@ def run_ours(args, rank, world, local_rank):
     phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
     gpu_index = phys[local_rank] if len(phys) > local_rank and phys[local_rank] else str(local_rank)
     with ClockSampler(gpu_index) as clk:
+        time.sleep(0.6)  # let nvidia-smi start sampling before the timed region
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
