@@ -117,6 +117,28 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
                         int variant, void* workspace, size_t workspace_bytes, int stages,
                         void* stream);
 
+/* Size of the fixed scratch array behind s2attn_bwd_noalloc_v (32 MiB). */
+#define S2_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* The backward (same arguments and results as s2attn_bwd_v) for callers that
+ * cannot allocate device memory, such as a plug-in inside a framework that
+ * owns the device heap, or a runtime held to a fixed memory footprint.  The
+ * pages describe no such entry point; it exists for those callers only.
+ * Instead of a caller-provided workspace it uses one file-scope device array
+ * of S2_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
+ * the process exits.  Shapes whose s2attn_bwd_workspace_size() exceeds that
+ * size are rejected with S2_ERR_UNSUPPORTED before anything is launched.
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it, so make that first call before any
+ * stream capture begins.  All calls share the one array: calls whose kernels
+ * overlap on the GPU (other streams, other host threads) race on it.  No
+ * allocating routine is called; the dq accumulator inside the array is
+ * cleared on every call. */
+int s2attn_bwd_noalloc_v(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
+                         int variant, void* stream);
+
 /* Debug: the (query, key) pairs the kernels visit for one head class
  * (0: heads [0,H/2), 1: heads [H/2,H); ignored for S2_DENSE_CAUSAL), computed
  * by the same scheduler and masks as the forward/backward kernels.

@@ -29,6 +29,8 @@ SIGNATURES = {
                       _int, _vp, _sz, _vp], _int),
     "s2attn_bwd_stages_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                              _int, _vp, _sz, _int, _vp], _int),
+    "s2attn_bwd_noalloc_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
+                              _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
@@ -117,6 +119,12 @@ def s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_vali
     return lib().s2attn_bwd_stages_v(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
                                      _ptr(dk), _ptr(dv), B, N, H, D, G, n_valid, variant, _ptr(workspace),
                                      workspace_bytes, stages, _stream(stream))
+
+
+def s2attn_bwd_noalloc_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_valid, variant, stream=None) -> int:
+    """Backward without a caller workspace (fixed library scratch; see include/s2attn.h)."""
+    return lib().s2attn_bwd_noalloc_v(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                                      _ptr(dk), _ptr(dv), B, N, H, D, G, n_valid, variant, _stream(stream))
 
 
 def s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, out, stream=None) -> int:

@@ -41,6 +41,9 @@ struct BwdArgs {
 int launch_fwd(const FwdArgs& a);
 // stages: 1 = prepare (Delta, lse2, zero accumulator), 2 = main, 4 = dq convert.
 int launch_bwd(const BwdArgs& a, int stages);
+// Sets the calling thread's s2attn_last_error() message; returns `code`.
+int report_error(int code, const char* fmt, ...);
+
 int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
 
 }  // namespace s2

@@ -135,6 +135,19 @@ int launch_status(int rc, const char* what) {
 
 }  // namespace
 
+namespace s2 {
+// Records a message for s2attn_last_error() from other translation units.
+int report_error(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+}  // namespace s2
+
 extern "C" {
 
 int s2attn_version(void) { return 100; }

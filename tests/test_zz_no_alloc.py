@@ -1,0 +1,54 @@
+"""The allocation-free backward entry point (needs a B200).
+
+s2attn_bwd_noalloc_v serves callers that cannot allocate device memory: it
+takes its scratch from a fixed array inside the library instead of a
+caller-provided workspace.  Its results must match s2attn_bwd_v (same
+tolerance as the other backward tests) on two calls in a row, the second one
+reusing whatever the first left in the shared array.  This file is collected
+last so that a failure here does not hide the other tests' results.
+"""
+from __future__ import annotations
+
+import pytest
+import torch
+
+from shifted_sparse_attention_b200 import binding as s2
+from shifted_sparse_attention_b200 import synthetic
+from tests.tolerance import check_grad
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("B,N,H,D,G,variant,nv", [
+    (2, 2048, 4, 128, 512, 0, 1900),
+    (1, 2048, 4, 128, 512, 1, None),
+    (1, 1024, 8, 64, 256, 0, None),
+])
+def test_noalloc_backward_matches_workspace_backward(B, N, H, D, G, variant, nv):
+    L = s2.lib()
+    n_valid = N if nv is None else nv
+    x = synthetic.draw(B, N, H, D, seed=77 + N + variant)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "dout"))
+    o, lse = s2.forward(q, k, v, G, variant, n_valid)
+    ref = s2.backward(q, k, v, o, do, lse, G, variant, n_valid)
+    stream = torch.cuda.current_stream().cuda_stream
+    for call in range(2):
+        dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
+        rc = L.s2attn_bwd_noalloc_v(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                                    lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                    B, N, H, D, G, n_valid, variant, stream)
+        assert rc == s2.S2_OK, s2.s2attn_last_error()
+        torch.cuda.synchronize()
+        s2.check_status()
+        for name, got, want in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            check_grad(name, got.float().cpu().numpy(), want.float().cpu().numpy(), "call %d" % call)
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    L = s2.lib()
+    B, N, H, D = 1, 32768, 32, 128  # needs ~513 MiB of scratch
+    assert s2.s2attn_bwd_workspace_size(B, N, H, D) > (32 << 20)
+    fake = 1 << 20  # never dereferenced: rejected before any launch
+    rc = L.s2attn_bwd_noalloc_v(*([fake] * 9), B, N, H, D, 8192, N, 0, None)
+    assert rc == s2.S2_ERR_UNSUPPORTED
+    assert "scratch" in s2.s2attn_last_error()
