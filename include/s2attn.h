@@ -80,8 +80,8 @@ int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* ls
                  void* stream);
 
 /* Bytes of device workspace s2attn_bwd needs: two float32 row statistics
- * ([B,H,N] each: Delta_i = dout_i·o_i and lse_i·log2(e)) and a float32 dq
- * accumulator ([B,N,H,D]), each part starting on a 256-byte boundary. */
+ * ([B,H,N] each, derived from Delta_i = dout_i·o_i and lse_i) and a float32
+ * dq accumulator ([B,N,H,D]), each part starting on a 256-byte boundary. */
 size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D);
 
 /* Backward.  Inputs q, k, v, o, dout (bf16), lse (fp32) as produced by the
@@ -102,8 +102,9 @@ int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, con
 /* The backward is three launches on `stream`; s2attn_bwd_v runs all of them
  * in order.  Running them one at a time (same arguments, `stages` a bit set)
  * lets a caller time or overlap them separately:
- *   S2_BWD_PREPARE  Delta_i = dout_i·o_i, lse_i·log2(e) and a zeroed dq
- *                   accumulator in the workspace (reads o, dout, lse);
+ *   S2_BWD_PREPARE  row statistics from Delta_i = dout_i·o_i and lse_i, and
+ *                   a zeroed dq accumulator, in the workspace (reads o,
+ *                   dout, lse);
  *   S2_BWD_MAIN     dk, dv, and the dq accumulator (reads q, k, v, dout and
  *                   the workspace written by the prepare stage);
  *   S2_BWD_FINISH   dq = bf16(accumulator / sqrt(D)).

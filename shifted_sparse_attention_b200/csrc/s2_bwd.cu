@@ -9,8 +9,8 @@
 // shift and reshape only permute gradients, which here is index math).
 //
 // Three kernels on the caller's stream:
-//   1. s2_bwd_pre: Delta_i = dout_i·o_i and lse_i·log2(e) (+inf on padded
-//      rows, which zeroes their probabilities), per [B, H, N].
+//   1. s2_bwd_pre: -Delta_i = -(dout_i·o_i) and -lse_i·log2(e) (-inf on
+//      padded rows, which zeroes their probabilities), per [B, H, N].
 //   2. s2_bwd_kernel: one CTA per 128-key tile of a segment, walking the
 //      query tiles from the diagonal to the segment's end:
 //        S^T  = K Q^T        (TMEM)            dP^T = V dO^T     (TMEM)
@@ -77,8 +77,9 @@ __device__ __forceinline__ int next_q(const Plan& p, const Unit& u, int qt) {
 }  // namespace bwd
 
 // ------------------------------------------------------------------ preprocess
-// kTpr = D/8 threads per (b, i, h) row, 8 bf16 (16 bytes) each:
-// Delta = dout·o (fp32), lse2 = lse·log2(e), +inf on padded rows.
+// kTpr = D/8 threads per (b, i, h) row, 8 bf16 (16 bytes) each.  Stores the
+// negated statistics the main kernel adds: -Delta = -(dout·o) and
+// -lse·log2(e) (-inf on padded rows, which zeroes their probabilities).
 template <int D>
 __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restrict__ o,
                                                    const __nv_bfloat16* __restrict__ dout,
@@ -110,8 +111,8 @@ __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restric
     const int i = (int)(bi % N), b = (int)(bi / N);
     const size_t at = ((size_t)b * H + h) * N + i;
     const bool valid = i < n_valid;
-    delta[at] = valid ? acc : 0.f;
-    lse2[at] = valid ? lse[at] * 1.4426950408889634f : INFINITY;
+    delta[at] = valid ? -acc : 0.f;
+    lse2[at] = valid ? -lse[at] * 1.4426950408889634f : -INFINITY;
   }
 }
 
@@ -325,9 +326,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
               const int i = 4 * g + t;
               const int col = col0 + i;
               const bool vis = (col >= lo) && (col < hi);
-              const float pr = vis ? ex2(fmaf(__uint_as_float(sv[32 * c + i]), p.scale_log2, -lsv[t])) : 0.f;
+              const float pr = vis ? ex2(fmaf(__uint_as_float(sv[32 * c + i]), p.scale_log2, lsv[t])) : 0.f;
               pv[t] = pr;
-              dsv[t] = pr * (__uint_as_float(dp[i]) - dlv[t]);
+              dsv[t] = pr * (__uint_as_float(dp[i]) + dlv[t]);
             }
             pp[2 * g] = pack_bf16(pv[0], pv[1]);
             pp[2 * g + 1] = pack_bf16(pv[2], pv[3]);
@@ -479,8 +480,8 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
     s2_bwd_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                         const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                        const Plan p, const float* __restrict__ delta, const float* __restrict__ lse2,
-                        float* __restrict__ dq_acc, int* __restrict__ status) {
+                        const __grid_constant__ CUtensorMap tmdQacc, const Plan p, const float* __restrict__ delta,
+                        const float* __restrict__ lse2, int* __restrict__ status) {
   using namespace bwds;
   using L = bwds::Layout;
   constexpr int kChunks = D / 64;
@@ -641,42 +642,51 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
     bool ok = true;
     int n = 0;
     if (kvalid) {
+      const bool key_tile_ragged = k0 + kTile > p.n_valid;
+      const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
       for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
         const int st = n % kStages;
         const int q0 = tile_orig(p, u, qt);
-        int lo, hi;
-        query_range(p, u, kt, qt, j, lo, hi);
-        // the stage's lse2 / Delta rows come with its Q/dO tiles
+        // masks are needed on the diagonal tile and on a key tile with padding;
+        // padded queries are zeroed by their -inf statistic
+        const bool masked = (qt == kt) || key_tile_ragged;
+        int lo = 0, hi = kTile;
+        if (masked) query_range(p, u, kt, qt, j, lo, hi);
+        // the stage's -lse2 / -Delta rows come with its Q/dO tiles
         ok = s2_wait(bar(QD_FULL + st), (n / kStages) & 1, abort_flag, status, 32);
         if (!ok) break;
         ok = s2_wait(bar(SP_FULL + x), n & 1, abort_flag, status, 32);
         if (!ok) break;
         tc_fence_after();
+        const float2* nl = reinterpret_cast<const float2*>(smem + L::kStat + st * L::kStatBytes) + 32 * x;
+        const float2* nd = nl + kTile / 2;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int col0 = 64 * x + 32 * c;  // first query (tile-local) of this chunk
+        for (int c = 0; c < 2; ++c) {  // 32 query columns per chunk
           uint32_t sv[32], dp[32];
           tmem_ld32(tS(x) + lane_off + 32 * c, sv);
           tmem_ld32(tDP(x) + lane_off + 32 * c, dp);
           tmem_wait_ld();
-          const float* lsv = reinterpret_cast<const float*>(smem + L::kStat + st * L::kStatBytes) + col0;
-          const float* dlv = lsv + kTile;
           uint32_t pp[16], dsp[16];
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            float pr[2], ds[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const int col = col0 + i + t;
-              const bool vis = (col >= lo) && (col < hi);
-              const float e = ex2(fmaf(__uint_as_float(sv[i + t]), p.scale_log2, -lsv[i + t]));
-              pr[t] = vis ? e : 0.f;
-              ds[t] = pr[t] * (__uint_as_float(dp[i + t]) - dlv[i + t]);
+          for (int i = 0; i < 16; ++i) {
+            // P = 2^(S·log2(e)/sqrt(D) - lse·log2(e)),  dS = P (dP - Delta), two columns at a time
+            const float2 a =
+                __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl[16 * c + i]);
+            float p0 = ex2(a.x), p1 = ex2(a.y);
+            if (masked) {
+              const int col = 64 * x + 32 * c + 2 * i;
+              p0 = (col >= lo && col < hi) ? p0 : 0.f;
+              p1 = (col + 1 >= lo && col + 1 < hi) ? p1 : 0.f;
             }
-            pp[i / 2] = pack_bf16(pr[0], pr[1]);
-            dsp[i / 2] = pack_bf16(ds[0], ds[1]);
+            const float2 d2 =
+                __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[16 * c + i]);
+            const float2 ds = __fmul2_rn(make_float2(p0, p1), d2);
+            pp[i] = pack_bf16(p0, p1);
+            dsp[i] = pack_bf16(ds.x, ds.y);
           }
+          // P^T (bf16 pairs) into dP^T_x columns [16c, 16c + 16), already read
           tmem_st16(tDP(x) + lane_off + 16 * c, pp);
+          // dS^T row j, queries [32c, 32c + 32): 16-byte pieces 4c..4c+3, 128-byte swizzle
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int piece = 4 * c + q;
@@ -688,26 +698,38 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(DS_READY + x));
-        // dQ^T_x: lane = d, columns = the half's 64 queries
+        // dQ^T_x (lane = d, columns = the half's 64 queries): into registers, then
+        // release the TMEM columns at once so the next S^T_x / dP^T_x can start
         ok = s2_wait(bar(DQ_FULL + x), n & 1, abort_flag, status, 32);
         if (!ok) break;
         tc_fence_after();
-        const int qfirst = q0 + 64 * x;
-        const int nq = p.n_valid - qfirst;  // valid queries of the half (may be <= 0 or > 64)
-#pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
-          uint32_t dq[32];
-          tmem_ld32(tS(x) + lane_off + 32 * c2, dq);
-          tmem_wait_ld();
-          float* dst = dq_acc + ((size_t)(row_base + qfirst + 32 * c2) * p.H + u.h) * D + j;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c2 + i < nq) atomicAdd(dst + (size_t)i * p.H * D, __uint_as_float(dq[i]));
-        }
+        uint32_t dq[64];
+        tmem_ld32(tS(x) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&dq[0]));
+        tmem_ld32(tS(x) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&dq[32]));
+        tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(DQ_FREE + x));
+        // add into the fp32 accumulator with bulk tensor reductions, staged in the
+        // dS^T_x buffer (free: dK_x and dQ_x have consumed it): 32 queries per round,
+        // four 32 x 32 boxes (one per 32 values of d)
+        const uint32_t stage_row = sdS(x) + (j / 32) * 4096 + (j % 32) * 4;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) st_shared_f32(stage_row + i * 128, __uint_as_float(dq[32 * r + i]));
+          fence_proxy_async_smem();
+          named_bar_sync(3 + x, 128);
+          if (j == 0) {
+            for (int b = 0; b < 4; ++b)
+              tma_reduce_add_3d(&tmdQacc, sdS(x) + b * 4096, 32 * b, u.h, row_base + q0 + 64 * x + 32 * r);
+            tma_store_commit();
+            tma_store_wait_read();
+          }
+          named_bar_sync(3 + x, 128);
+        }
         ++n;
       }
+      if (j == 0) tma_store_wait_all();  // every reduction has landed before the CTA retires
     }
     // ---------------------------------------------------------- epilogue: dK, dV
     bool have = kvalid && ok && n > 0;
@@ -787,7 +809,7 @@ int launch_bwd_impl(const BwdArgs& a, int stages) {
       e = cudaFuncSetAttribute(s2_bwd_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwds::Layout::kBytes);
       if (e != cudaSuccess) return (int)e;
       s2_bwd_split_kernel<<<grid, bwds::kThreads, bwds::Layout::kBytes, a.stream>>>(
-          *a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK, *a.tmdV, p, a.delta, a.lse2, a.dq_acc, a.status);
+          *a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK, *a.tmdV, *a.tmdQacc, p, a.delta, a.lse2, a.status);
     } else {
       e = cudaFuncSetAttribute(s2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
       if (e != cudaSuccess) return (int)e;

@@ -26,12 +26,13 @@ struct BwdArgs {
   const CUtensorMap* tmdO;
   const CUtensorMap* tmdK;
   const CUtensorMap* tmdV;
+  const CUtensorMap* tmdQacc;  // fp32 dq accumulator, box 32 x 1 x 32, no swizzle
   Plan plan;
   const void* o;      // bf16 [B, N, H, D]
   const void* dout;   // bf16 [B, N, H, D]
   const float* lse;   // [B, H, N]
-  float* delta;       // workspace [B, H, N]: dout_i·o_i
-  float* lse2;        // workspace [B, H, N]: lse_i·log2(e), +inf on padded rows
+  float* delta;       // workspace [B, H, N]: -(dout_i·o_i)
+  float* lse2;        // workspace [B, H, N]: -lse_i·log2(e), -inf on padded rows
   float* dq_acc;      // workspace [B, N, H, D] fp32
   void* dq;           // bf16 [B, N, H, D]
   int* status;

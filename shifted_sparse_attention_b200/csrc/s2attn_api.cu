@@ -128,6 +128,19 @@ int make_tmap(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int6
   return S2_OK;
 }
 
+// The fp32 dq accumulator [B*N, H, D] for bulk reductions: box = 32 columns x 1 head x 32 rows.
+int make_tmap_acc(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t H, int64_t D) {
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(B * N)};
+  cuuint64_t strides[2] = {(cuuint64_t)(D * 4), (cuuint64_t)(H * D * 4)};
+  cuuint32_t box[3] = {32, 1, 32};
+  cuuint32_t elem[3] = {1, 1, 1};
+  CUresult r = st->encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(S2_ERR_CUDA, "cuTensorMapEncodeTiled (accumulator) failed (%d)", (int)r);
+  return S2_OK;
+}
+
 int launch_status(int rc, const char* what) {
   if (rc == 0) return S2_OK;
   return fail(S2_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString((cudaError_t)rc));
@@ -226,6 +239,9 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
   a.delta = static_cast<float*>(workspace);
   a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
   a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * sb);
+  CUtensorMap tacc;
+  if ((rc = make_tmap_acc(st, &tacc, a.dq_acc, B, N, H, D))) return rc;
+  a.tmdQacc = &tacc;
   a.dq = dq;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
