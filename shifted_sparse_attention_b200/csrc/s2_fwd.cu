@@ -91,10 +91,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto bar = [&](int i) { return smem_u32(&bars[i]); };
-  auto sQ = [&](int x) { return sb + L::kQ + x * L::kQBytes; };
-  auto sKV = [&](int slot) { return sb + L::kKV + slot * L::kKVBytes; };
-  auto sP = [&](int x) { return sb + L::kP + x * L::kPBytes; };
+  // Addresses are plain values (macros, #undef'd after the kernel): no lambda
+  // captures, so nothing the MMA issuer needs lives in memory.
+  const uint32_t sbar = smem_u32(bars);
+#define bar(i) (sbar + 8u * (uint32_t)(i))
+#define sQ(x) (sb + L::kQ + (uint32_t)(x) * L::kQBytes)
+#define sKV(slot) (sb + L::kKV + (uint32_t)(slot) * L::kKVBytes)
+#define sP(x) (sb + L::kP + (uint32_t)(x) * L::kPBytes)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
@@ -170,21 +173,26 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     if (lane == 0 && u.kmax >= 0) {
       constexpr uint32_t idesc_qk = umma_idesc_bf16(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = umma_idesc_bf16(128, D, 0, 1);
-      auto issue_qk = [&](int x, int slot) {
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-          umma_ss(tmem + x * 128, umma_desc_sw128(sQ(x) + off, 16, 1024),
-                  umma_desc_sw128(sKV(slot) + off, 16, 1024), idesc_qk, kk > 0);
-        }
-      };
-      auto issue_pv = [&](int x, int slot, bool acc) {
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint32_t aoff = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-          umma_ss(tmem + 256 + x * D, umma_desc_sw128(sP(x) + aoff, 16, 1024),
-                  umma_desc_sw128(sKV(slot) + kk * 2048, kChunkBytes, 1024), idesc_pv,
-                  (acc || kk > 0) ? 1u : 0u);
-        }
-      };
+      // Descriptors are built once per group and advanced by compile-time
+      // offsets (in 16-byte units): issuing an MMA then costs a 64-bit add.
+#define ISSUE_QK(x, slot)                                                                         \
+  do {                                                                                            \
+    const uint64_t a0_ = umma_desc_sw128(sQ(x), 16, 1024), b0_ = umma_desc_sw128(sKV(slot), 16, 1024); \
+    _Pragma("unroll") for (int kk = 0; kk < D / 16; ++kk) {                                       \
+      const uint64_t off_ = ((kk / 4) * kChunkBytes + (kk % 4) * 32) >> 4;                        \
+      umma_ss(tmem + (x) * 128, a0_ + off_, b0_ + off_, idesc_qk, kk > 0);                         \
+    }                                                                                             \
+  } while (0)
+#define ISSUE_PV(x, slot, acc)                                                                    \
+  do {                                                                                            \
+    const uint64_t a0_ = umma_desc_sw128(sP(x), 16, 1024);                                        \
+    const uint64_t b0_ = umma_desc_sw128(sKV(slot), kChunkBytes, 1024);                           \
+    _Pragma("unroll") for (int kk = 0; kk < kTile / 16; ++kk) {                                   \
+      const uint64_t aoff_ = ((kk / 4) * kChunkBytes + (kk % 4) * 32) >> 4;                        \
+      umma_ss(tmem + 256 + (x) * D, a0_ + aoff_, b0_ + (uint64_t)(kk * 2048 >> 4), idesc_pv,      \
+              ((acc) || kk > 0) ? 1u : 0u);                                                       \
+    }                                                                                             \
+  } while (0)
       bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
       int nqk[2] = {0, 0}, npv[2] = {0, 0};
       int e = 0;
@@ -195,7 +203,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         tc_fence_after();
         for (int x = 0; ok && x < 2; ++x)
           if (tile_takes(p, u, x, kc)) {
-            issue_qk(x, eK % kSlots);
+            ISSUE_QK(x, eK % kSlots);
             umma_commit(bar(S_FULL + x));
             ++nqk[x];
           }
@@ -215,7 +223,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             if (nqk[x] > 0) ok = s2_wait(bar(S_FREE + x), (nqk[x] - 1) & 1, abort_flag, status, 2);
             if (!ok) break;
             tc_fence_after();
-            issue_qk(x, eK % kSlots);
+            ISSUE_QK(x, eK % kSlots);
             umma_commit(bar(S_FULL + x));
             ++nqk[x];
           }
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             ok = s2_wait(bar(P_FULL + x), npv[x] & 1, abort_flag, status, 2);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(x, eV % kSlots, npv[x] > 0);
+            ISSUE_PV(x, eV % kSlots, npv[x] > 0);
             umma_commit(bar(PV_DONE + x));
             ++npv[x];
           }
@@ -376,6 +384,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     tmem_dealloc(tmem, 512);
   }
 }
+
+#undef ISSUE_QK
+#undef ISSUE_PV
+#undef bar
+#undef sQ
+#undef sKV
+#undef sP
 
 template <int D>
 int launch_fwd_impl(const FwdArgs& a) {
