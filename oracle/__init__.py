@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
         L.s2o_attention.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, i64,
                                     ctypes.c_int, i64, i64, i64p, i64, dp, dp, dp, dp, dp]
         L.s2o_attention.restype = ctypes.c_int
+        L.s2o_attention_window.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, i64,
+                                           ctypes.c_int, i64, i64, i64p, i64, dp, dp, dp, dp, dp]
+        L.s2o_attention_window.restype = ctypes.c_int
         L.s2o_num_threads.argtypes = []
         L.s2o_num_threads.restype = ctypes.c_int
         _lib = L
@@ -151,6 +154,41 @@ def attention(q, k, v, dout=None, *, G: int, variant: int, n_valid: int | None =
         _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
         _ptr(gb, ctypes.c_uint16) if want_bwd else None,
         B, N, H, D, G, nv, variant, r0, r1, hp, nh,
+        _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
+        _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double),
+    )
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments (rc=%d)" % rc)
+    out = {"o": o, "lse": lse}
+    if want_bwd:
+        out.update(dq=dq, dk=dk, dv=dv)
+    return out
+
+
+def attention_window(q, k, v, dout=None, *, G: int, variant: int, rows: tuple[int, int], heads,
+                     n_valid: int | None = None):
+    """The oracle on query rows [r0, r1) of the given heads (flattened b*H+h),
+    with compact outputs: o, dq, dk, dv [len(heads), r1 - r0, D]; lse
+    [len(heads), r1 - r0].  dk / dv hold the contributions of the window's rows
+    to the window's keys only (exact for keys whose visible-from rows all lie in
+    the window)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, N, H, D = qb.shape
+    nv = N if n_valid is None else int(n_valid)
+    r0, r1 = rows
+    harr = np.ascontiguousarray(np.asarray(heads, dtype=np.int64))
+    nh, W = len(harr), r1 - r0
+    o = np.full((nh, W, D), np.nan)
+    lse = np.full((nh, W), np.nan)
+    want_bwd = dout is not None
+    gb = _bits(dout) if want_bwd else None
+    dq = np.full((nh, W, D), np.nan) if want_bwd else np.zeros(1)
+    dk = np.zeros((nh, W, D)) if want_bwd else np.zeros(1)
+    dv = np.zeros((nh, W, D)) if want_bwd else np.zeros(1)
+    rc = lib().s2o_attention_window(
+        _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
+        _ptr(gb, ctypes.c_uint16) if want_bwd else None,
+        B, N, H, D, G, nv, variant, r0, r1, _ptr(harr, ctypes.c_int64), nh,
         _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
         _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double),
     )

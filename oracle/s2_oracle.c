@@ -226,6 +226,100 @@ int s2o_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const
   return 0;
 }
 
+/*
+ * The same computation on a window of query rows [r0, r1) of selected heads,
+ * with compact outputs (for large inputs whose full-size float64 outputs
+ * would not fit in memory):
+ *   o_w, dq_w  [n_heads][r1 - r0][D]   rows r0..r1-1
+ *   lse_w      [n_heads][r1 - r0]
+ *   dk_w, dv_w [n_heads][r1 - r0][D]   keys r0..r1-1, ACCUMULATED from the
+ *              window's rows only (exact for keys whose visible-from rows
+ *              all lie inside the window; the caller zeroes them)
+ * heads: flattened (b*H + h) list.  dout may be NULL (forward only).
+ */
+int s2o_attention_window(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                         int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
+                         int variant, int64_t r0, int64_t r1, const int64_t* heads, int64_t n_heads,
+                         double* o_w, double* lse_w, double* dq_w, double* dk_w, double* dv_w) {
+  if (B < 1 || N < 1 || H < 2 || D < 1 || G < 2 || (H % 2) || (G % 2) || (N % G)) return -1;
+  if (n_valid < 0 || n_valid > N || r0 < 0 || r1 > N || r0 > r1 || !heads) return -1;
+  if (variant < 0 || variant > 2) return -1;
+  const double scale = 1.0 / sqrt((double)D);
+  const int64_t W = r1 - r0;
+
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < n_heads; ++t) {
+    const int64_t bh = heads[t];
+    const int64_t b = bh / H, h = bh % H;
+    const int head_class = (h >= H / 2) ? 1 : 0;
+    double* qi = (double*)malloc(sizeof(double) * D);
+    double* gi = (double*)malloc(sizeof(double) * D);
+    double* oi = (double*)malloc(sizeof(double) * D);
+    double* dqi = (double*)malloc(sizeof(double) * D);
+    double* z = (double*)malloc(sizeof(double) * N);
+    int64_t* js = (int64_t*)malloc(sizeof(int64_t) * N);
+    for (int64_t i = r0; i < r1; ++i) {
+      const size_t wi = (size_t)(t * W + (i - r0));
+      int64_t ns = 0;
+      for (int64_t j = 0; j < N; ++j)
+        if (s2o_visible(N, G, n_valid, variant, head_class, i, j)) js[ns++] = j;
+      for (int64_t d = 0; d < D; ++d) qi[d] = bf16_to_double(q[at(N, H, D, b, i, h, d)]);
+      if (ns == 0) {
+        for (int64_t d = 0; d < D; ++d) {
+          o_w[wi * D + d] = 0.0;
+          if (dout) dq_w[wi * D + d] = 0.0;
+        }
+        lse_w[wi] = -INFINITY;
+        continue;
+      }
+      double m = -INFINITY;
+      for (int64_t t2 = 0; t2 < ns; ++t2) {
+        const int64_t j = js[t2];
+        double acc = 0.0;
+        for (int64_t d = 0; d < D; ++d) acc += qi[d] * bf16_to_double(k[at(N, H, D, b, j, h, d)]);
+        z[t2] = scale * acc;
+        if (z[t2] > m) m = z[t2];
+      }
+      double l = 0.0;
+      for (int64_t t2 = 0; t2 < ns; ++t2) l += exp(z[t2] - m);
+      for (int64_t d = 0; d < D; ++d) oi[d] = 0.0;
+      for (int64_t t2 = 0; t2 < ns; ++t2) {
+        const double p = exp(z[t2] - m) / l;
+        const int64_t j = js[t2];
+        for (int64_t d = 0; d < D; ++d) oi[d] += p * bf16_to_double(v[at(N, H, D, b, j, h, d)]);
+      }
+      const double lse_i = m + log(l);
+      for (int64_t d = 0; d < D; ++d) o_w[wi * D + d] = oi[d];
+      lse_w[wi] = lse_i;
+      if (!dout) continue;
+      for (int64_t d = 0; d < D; ++d)
+        gi[d] = (i < n_valid) ? bf16_to_double(dout[at(N, H, D, b, i, h, d)]) : 0.0;
+      double delta = 0.0;
+      for (int64_t d = 0; d < D; ++d) delta += gi[d] * oi[d];
+      for (int64_t d = 0; d < D; ++d) dqi[d] = 0.0;
+      for (int64_t t2 = 0; t2 < ns; ++t2) {
+        const int64_t j = js[t2];
+        const double a = exp(z[t2] - lse_i);
+        double gv = 0.0;
+        for (int64_t d = 0; d < D; ++d) gv += gi[d] * bf16_to_double(v[at(N, H, D, b, j, h, d)]);
+        const double ds = a * (gv - delta);
+        const int in_window = (j >= r0 && j < r1);
+        const size_t wj = (size_t)(t * W + (j - r0));
+        for (int64_t d = 0; d < D; ++d) {
+          dqi[d] += scale * ds * bf16_to_double(k[at(N, H, D, b, j, h, d)]);
+          if (in_window) {
+            dk_w[wj * D + d] += scale * ds * qi[d];
+            dv_w[wj * D + d] += a * gi[d];
+          }
+        }
+      }
+      for (int64_t d = 0; d < D; ++d) dq_w[wi * D + d] = dqi[d];
+    }
+    free(qi); free(gi); free(oi); free(dqi); free(z); free(js);
+  }
+  return 0;
+}
+
 /* Number of threads the OpenMP runtime will use for s2o_attention. */
 int s2o_num_threads(void) {
 #ifdef _OPENMP

@@ -324,6 +324,28 @@ def test_row_window_and_head_subset_compose_to_full_result():
                                        full[name][b, :, h], atol=1e-13, rtol=0)
 
 
+@pytest.mark.parametrize("variant", [STRICT, ROLLED, DENSE])
+def test_window_entry_equals_full_oracle(variant):
+    # the windowed entry (used for full-size samples) against the pinned full routine
+    B, N, H, D, G, nv = 2, 48, 4, 8, 12, 43
+    x = synthetic.draw(B, N, H, D, seed=31)
+    full = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, n_valid=nv)
+    heads = [0, 3, 5, 6]
+    for r0, r1 in ((0, 48), (18, 24), (36, 48)):
+        w = oracle.attention_window(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, rows=(r0, r1),
+                                    heads=heads, n_valid=nv)
+        part = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, n_valid=nv,
+                                rows=(r0, r1), heads=heads)
+        for t, bh in enumerate(heads):
+            b, h = divmod(bh, H)
+            np.testing.assert_array_equal(w["o"][t], full["o"][b, r0:r1, h])
+            np.testing.assert_array_equal(w["lse"][t], full["lse"][b, h, r0:r1])
+            np.testing.assert_array_equal(w["dq"][t], full["dq"][b, r0:r1, h])
+            # dk, dv: the window's rows' contributions to the window's keys
+            np.testing.assert_allclose(w["dk"][t], part["dk"][b, r0:r1, h], rtol=0, atol=1e-15)
+            np.testing.assert_allclose(w["dv"][t], part["dv"][b, r0:r1, h], rtol=0, atol=1e-15)
+
+
 # --------------------------------------------------------------------------
 # power of the pins: plausible mistakes in the predicate must be rejected
 

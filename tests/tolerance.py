@@ -43,9 +43,13 @@ def check_o(o_gpu, o_ref, where: str = "") -> dict:
     return stats
 
 
-def check_grad(name, g_gpu, g_ref, where: str = "") -> dict:
+def check_grad(name, g_gpu, g_ref, where: str = "", tensor_max: float | None = None) -> dict:
+    """tensor_max: max |x| of the whole gradient tensor when g_* are a sample of it
+    (the bound is scaled by the tensor's max-norm); defaults to the sample's own."""
     g_gpu, g_ref = to_np(g_gpu), np.asarray(g_ref)
     scale = np.abs(g_ref).max()
+    if tensor_max is not None:
+        scale = max(scale, float(tensor_max))
     scale = scale if scale > 0 else 1.0
     err = np.abs(g_gpu - g_ref) / scale
     stats = dict(max_rel=float(err.max()), mean_rel=float(err.mean()))
