@@ -457,7 +457,8 @@ enum Bar {
   DQ_FULL = 9,    // + half (2)
   DQ_FREE = 11,   // + half (2)
   ACC_DONE = 13,
-  NUM_BARS = 14
+  RED_DONE = 14,  // + stage (2): both halves' dQ reductions have read their staging rows
+  NUM_BARS = 16
 };
 
 struct Layout {
@@ -522,6 +523,7 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
       mbar_init(bar(DS_READY + i), 128);
       mbar_init(bar(DQ_FULL + i), 1);
       mbar_init(bar(DQ_FREE + i), 128);
+      mbar_init(bar(RED_DONE + i), 2);
     }
     mbar_init(bar(ACC_DONE), 1);
     *abort_flag = 0;
@@ -556,7 +558,10 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
       bool ok = true;
       for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
         const int st = n % kStages;
-        if (n >= kStages) ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
+        if (n >= kStages) {  // MMAs done with the stage, and the dQ reductions staged in it have read it
+          ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
+          if (ok) ok = s2_wait(bar(RED_DONE + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
+        }
         if (!ok) break;
         mbar_arrive_expect_tx(bar(QD_FULL + st), 2 * L::kTileBytes + L::kStatBytes);
         const int q0 = tile_orig(p, u, qt);
@@ -709,28 +714,35 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(bar(DQ_FREE + x));
-        // add into the fp32 accumulator with bulk tensor reductions, staged in the
-        // dS^T_x buffer (free: dK_x and dQ_x have consumed it): 32 queries per round,
-        // four 32 x 32 boxes (one per 32 values of d)
-        const uint32_t stage_row = sdS(x) + (j / 32) * 4096 + (j % 32) * 4;
+        // Add into the fp32 accumulator with bulk tensor reductions, staged in this
+        // half's rows [64x, 64x + 64) of the stage's Q and dO tiles: every MMA
+        // reading them (S^T_x, dP^T_x, dV_x, dK_x) has completed at DQ_FULL[x], the
+        // other half never reads them, and the producer refills the stage only
+        // after RED_DONE.  Four 8 KB regions (Q and dO, 64-column chunks 0 and 1)
+        // hold the eight 32 x 32 fp32 boxes: region b = d / 32, box row = query.
+        const uint32_t region = ((j / 32) < 2 ? sQ(st) : sdO(st)) + ((j / 32) & 1) * kChunkBytes + x * 8192;
+        const uint32_t stage_col = region + (j % 32) * 4;
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) st_shared_f32(stage_row + i * 128, __uint_as_float(dq[32 * r + i]));
-          fence_proxy_async_smem();
-          named_bar_sync(3 + x, 128);
-          if (j == 0) {
-            for (int b = 0; b < 4; ++b)
-              tma_reduce_add_3d(&tmdQacc, sdS(x) + b * 4096, 32 * b, u.h, row_base + q0 + 64 * x + 32 * r);
-            tma_store_commit();
-            tma_store_wait_read();
+        for (int q = 0; q < 64; ++q)
+          st_shared_f32(stage_col + (q / 32) * 4096 + (q % 32) * 128, __uint_as_float(dq[q]));
+        fence_proxy_async_smem();
+        named_bar_sync(3 + x, 128);
+        if (j == 0) {
+          for (int b = 0; b < 4; ++b) {
+            const uint32_t reg = (b < 2 ? sQ(st) : sdO(st)) + (b & 1) * kChunkBytes + x * 8192;
+            for (int r = 0; r < 2; ++r)
+              tma_reduce_add_3d(&tmdQacc, reg + r * 4096, 32 * b, u.h, row_base + q0 + 64 * x + 32 * r);
           }
-          named_bar_sync(3 + x, 128);
+          tma_store_commit();
+          tma_store_wait_read();
+          mbar_arrive(bar(RED_DONE + st));
         }
         ++n;
       }
       if (j == 0) tma_store_wait_all();  // every reduction has landed before the CTA retires
     }
+    // the last reductions read Q stage rows the epilogue below overwrites
+    named_bar_sync(1, 256);
     // ---------------------------------------------------------- epilogue: dK, dV
     bool have = kvalid && ok && n > 0;
     if (have) {

@@ -19,7 +19,7 @@
 // are 128-byte-swizzled, 1024-byte aligned, as TMA writes and UMMA reads them.
 // MMA order per key tile k (software pipelined so that the tensor core works
 // on the next S while the softmax warps exponentiate the current one):
-//     S_A(k+1)=Q_A K(k+1)^T, O_A += P_A(k) V(k), S_B(k+1)=Q_B K(k+1)^T, O_B += P_B(k) V(k)
+//     S_A(k+1)=Q_A K(k+1)^T, S_B(k+1)=Q_B K(k+1)^T, O_A += P_A(k) V(k), O_B += P_B(k) V(k)
 // Softmax uses base-2 exponentials with a lazily updated running max: O and
 // l are rescaled only when the row max grows by more than 8 (a factor 256),
 // which keeps bf16 P and fp32 sums exact enough and skips most rescales.
@@ -218,7 +218,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           if (!ok) break;
           tc_fence_after();
         }
-        for (int x = 0; x < 2; ++x) {
+        // Both next-tile score MMAs first, then both PV MMAs: a late P on one
+        // query tile never holds back the other tile's next S.
+        for (int x = 0; x < 2 && ok; ++x) {
           if (kn >= 0 && tile_takes(p, u, x, kn)) {
             if (nqk[x] > 0) ok = s2_wait(bar(S_FREE + x), (nqk[x] - 1) & 1, abort_flag, status, 2);
             if (!ok) break;
@@ -227,12 +229,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             umma_commit(bar(S_FULL + x));
             ++nqk[x];
           }
-          if (x == 1 && kn >= 0) umma_commit(bar(KV_EMPTY + eK % kSlots));
+        }
+        if (!ok) break;
+        if (kn >= 0) umma_commit(bar(KV_EMPTY + eK % kSlots));
+        ok = s2_wait(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
+        for (int x = 0; x < 2 && ok; ++x) {
           if (tile_takes(p, u, x, kc)) {
-            if (x == 0 || !tile_takes(p, u, 0, kc)) {
-              ok = s2_wait(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
-              if (!ok) break;
-            }
             ok = s2_wait(bar(P_FULL + x), npv[x] & 1, abort_flag, status, 2);
             if (!ok) break;
             tc_fence_after();
@@ -277,11 +279,24 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           tc_fence_before();
           mbar_arrive(bar(S_FREE + x));
 
+          // Masks (the causal triangle of the diagonal tile, padded keys or rows)
+          // only where some row of the warp needs them.
           const int lim = col_limit(p, u, u.t[x], k, r);
-          float mx = -INFINITY;
+          if (!__all_sync(0xffffffffu, lim == kTile)) {
 #pragma unroll
-          for (int c = 0; c < kTile; ++c)
-            if (c < lim) mx = fmaxf(mx, __uint_as_float(s[c]) * p.scale_log2);
+            for (int c = 0; c < kTile; ++c)
+              if (c >= lim) s[c] = 0xff800000u;  // -inf
+          }
+          // Row max as a 4-way tree of 3-input max (short dependency chains), then
+          // scaled once (scale > 0 keeps the order).
+          float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < kTile; c += 8) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mq[q] = fmax3(mq[q], __uint_as_float(s[c + 2 * q]), __uint_as_float(s[c + 2 * q + 1]));
+          }
+          const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * p.scale_log2;
           const float m_new = fmaxf(m_used, mx);
           const bool need = m_new > m_used + 8.0f;
           float factor = 1.f;
@@ -291,19 +306,22 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             m_used = m_new;
           }
           const float m_exp = (m_used == -INFINITY) ? 0.f : m_used;
-          // p = 2^(x - m), rounded to bf16 pairs in place (s[c/2] <- pair c, c+1);
-          // l sums the ROUNDED weights, so o = sum p~ v / sum p~ stays a convex
-          // combination of the v_j whatever the rounding of each p.
-          float sum = 0.f;
+          // p = 2^(x·c - m) two columns at a time, rounded to bf16 pairs in place
+          // (s[c/2] <- pair c, c+1); l sums the ROUNDED weights in four packed
+          // accumulators, so o = sum p~ v / sum p~ stays a convex combination of the v_j.
+          const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 nm2 = make_float2(-m_exp, -m_exp);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < kTile; c += 2) {
-            const float e0 = (c < lim) ? ex2(fmaf(__uint_as_float(s[c]), p.scale_log2, -m_exp)) : 0.f;
-            const float e1 = (c + 1 < lim) ? ex2(fmaf(__uint_as_float(s[c + 1]), p.scale_log2, -m_exp)) : 0.f;
-            const uint32_t pk = pack_bf16(e0, e1);
+            const float2 a = __ffma2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])), c2, nm2);
+            const uint32_t pk = pack_bf16(ex2(a.x), ex2(a.y));
             s[c / 2] = pk;
-            sum += __uint_as_float(pk << 16) + __uint_as_float(pk & 0xffff0000u);
+            acc[(c / 2) & 3] = __fadd2_rn(acc[(c / 2) & 3], make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xffff0000u)));
           }
-          l += sum;
+          const float2 acc01 = __fadd2_rn(acc[0], acc[1]), acc23 = __fadd2_rn(acc[2], acc[3]);
+          const float2 acct = __fadd2_rn(acc01, acc23);
+          l += acct.x + acct.y;
 
           if (n > 0) {
             ok = s2_wait(bar(PV_DONE + x), (n - 1) & 1, abort_flag, status, 4);
