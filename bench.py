@@ -3,8 +3,8 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
 
 One step = one pass of the whole hot path over one batch: s2attn_fwd, then
-the three backward stages (prepare, main, dq finish), on inputs resident in
-HBM.  Default workload: B=1, H=32, N=32768, D=128, G=8192, strict variant,
+the three backward stages (prepare, dK/dV pass, dQ pass), on inputs resident
+in HBM.  Default workload: B=1, H=32, N=32768, D=128, G=8192, strict variant,
 bf16 Q/K/V/dO ~ N(0,1) with K doubled on 5% of positions.
 
 Metric: useful causal TFLOP/s = 7·B·H·N·G·D per step (forward 2·B·H·N·G·D,
@@ -291,10 +291,10 @@ def run_ours(args, rank, world, local_rank):
         s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE)
         if ev is not None:
             ev[2].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_MAIN)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DKDV)
         if ev is not None:
             ev[3].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_FINISH)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ)
         if ev is not None:
             ev[4].record(stream)
 
@@ -322,7 +322,7 @@ def run_ours(args, rank, world, local_rank):
     s2.check_status()
     ms = start.elapsed_time(end)
     per = {name: sum(e[a].elapsed_time(e[b]) for e in evs) / args.steps
-           for name, a, b in (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_main", 2, 3), ("bwd_finish", 3, 4))}
+           for name, a, b in (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_dkdv", 2, 3), ("bwd_dq", 3, 4))}
     clocks = clk.summary()
 
     # e2e: the same step through the public API from pinned host buffers, copies included
@@ -384,13 +384,16 @@ def run_ours(args, rank, world, local_rank):
         pairs = w.B * (w.H // 2) * (pc[0] + pc[1])
     else:
         pairs = None
-    # dominant kernel: the longer of the forward and the backward main kernel
-    dom = "bwd_main" if per["bwd_main"] >= per["fwd"] else "fwd"
-    per_pair = {"fwd": 4 * D, "bwd_main": 10 * D}[dom]
-    algo = pairs * per_pair if pairs is not None else w.formula_flops(passes="fwd" if dom == "fwd" else "bwd")
+    # dominant kernel: the longest of the forward, the dK/dV pass and the dQ pass.
+    # Algorithmic FLOPs per visited pair: forward 4·D (Q K^T, P V); dK/dV pass
+    # 8·D (S, dP, dV, dK); dQ pass 2·D (dQ only: its S and dP are recomputed).
+    dom = max(("fwd", "bwd_dkdv", "bwd_dq"), key=lambda k: per[k])
+    per_pair = {"fwd": 4 * D, "bwd_dkdv": 8 * D, "bwd_dq": 2 * D}[dom]
+    share = {"fwd": 1.0, "bwd_dkdv": 0.8, "bwd_dq": 0.2}[dom]
+    algo = pairs * per_pair if pairs is not None else share * w.formula_flops(passes="fwd" if dom == "fwd" else "bwd")
     achieved = algo / (per[dom] * 1e-3) / 1e12
-    src = {"fwd": "s2_fwd.cu", "bwd_main": "s2_bwd.cu"}[dom]
-    kname = {"fwd": "s2_fwd_kernel", "bwd_main": "s2_bwd_split_kernel" if D == 128 else "s2_bwd_kernel"}[dom]
+    src = {"fwd": "s2_fwd.cu", "bwd_dkdv": "s2_bwd.cu", "bwd_dq": "s2_bwd.cu"}[dom]
+    kname = {"fwd": "s2_fwd_kernel", "bwd_dkdv": "s2_bwd_dkdv_kernel", "bwd_dq": "s2_bwd_dq_kernel"}[dom]
     roof = {"bound": "tensor", "kernel": kname,
             "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
             "frac": achieved / pk["bf16_sustained"],

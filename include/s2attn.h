@@ -80,8 +80,8 @@ int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* ls
                  void* stream);
 
 /* Bytes of device workspace s2attn_bwd needs: two float32 row statistics
- * ([B,H,N] each, derived from Delta_i = dout_i·o_i and lse_i) and a float32
- * dq accumulator ([B,N,H,D]), each part starting on a 256-byte boundary. */
+ * ([B,H,N] each, derived from Delta_i = dout_i·o_i and lse_i), each starting on
+ * a 256-byte boundary.  D does not enter the size. */
 size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D);
 
 /* Backward.  Inputs q, k, v, o, dout (bf16), lse (fp32) as produced by the
@@ -102,15 +102,15 @@ int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, con
 /* The backward is three launches on `stream`; s2attn_bwd_v runs all of them
  * in order.  Running them one at a time (same arguments, `stages` a bit set)
  * lets a caller time or overlap them separately:
- *   S2_BWD_PREPARE  row statistics from Delta_i = dout_i·o_i and lse_i, and
- *                   a zeroed dq accumulator, in the workspace (reads o,
- *                   dout, lse);
- *   S2_BWD_MAIN     dk, dv, and the dq accumulator (reads q, k, v, dout and
- *                   the workspace written by the prepare stage);
- *   S2_BWD_FINISH   dq = bf16(accumulator / sqrt(D)).
- * A stage assumes the earlier stages of the same call sequence have run on
- * the same stream with the same workspace. */
-enum { S2_BWD_PREPARE = 1, S2_BWD_MAIN = 2, S2_BWD_FINISH = 4, S2_BWD_ALL = 7 };
+ *   S2_BWD_PREPARE  row statistics from Delta_i = dout_i·o_i and lse_i, in the
+ *                   workspace (reads o, dout, lse);
+ *   S2_BWD_DKDV     dk and dv (reads q, k, v, dout and the workspace);
+ *   S2_BWD_DQ       dq (reads q, k, v, dout and the workspace).
+ * The dk/dv and dq stages are independent of each other; both need the
+ * prepare stage of the same call sequence to have run on the same stream
+ * with the same workspace.  dq is bitwise reproducible; no stage uses
+ * atomic accumulation. */
+enum { S2_BWD_PREPARE = 1, S2_BWD_DKDV = 2, S2_BWD_DQ = 4, S2_BWD_ALL = 7 };
 
 int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o,
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
@@ -133,8 +133,8 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
  * that device current) and caches it, so make that first call before any
  * stream capture begins.  All calls share the one array: calls whose kernels
  * overlap on the GPU (other streams, other host threads) race on it.  No
- * allocating routine is called; the dq accumulator inside the array is
- * cleared on every call. */
+ * allocating routine is called; every call rewrites the statistics it reads
+ * before reading them. */
 int s2attn_bwd_noalloc_v(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
                          int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
@@ -158,7 +158,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor). */
+/* ABI version of this header (major*100 + minor): 101. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

@@ -111,7 +111,7 @@ def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, variant, worksp
                             _ptr(dv), B, N, H, D, G, variant, _ptr(workspace), workspace_bytes, _stream(stream))
 
 
-S2_BWD_PREPARE, S2_BWD_MAIN, S2_BWD_FINISH, S2_BWD_ALL = 1, 2, 4, 7
+S2_BWD_PREPARE, S2_BWD_DKDV, S2_BWD_DQ, S2_BWD_ALL = 1, 2, 4, 7
 
 
 def s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,

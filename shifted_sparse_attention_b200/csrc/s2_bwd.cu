@@ -8,22 +8,24 @@
 // Only in-group pairs are ever computed (§1: the backward stays sparse; the
 // shift and reshape only permute gradients, which here is index math).
 //
-// Three kernels on the caller's stream:
+// Three launches on the caller's stream:
 //   1. s2_bwd_pre: -Delta_i = -(dout_i·o_i) and -lse_i·log2(e) (-inf on
 //      padded rows, which zeroes their probabilities), per [B, H, N].
-//   2. s2_bwd_kernel: one CTA per 128-key tile of a segment, walking the
-//      query tiles from the diagonal to the segment's end:
-//        S^T  = K Q^T        (TMEM)            dP^T = V dO^T     (TMEM)
-//        P^T  = exp2(S^T·c - lse2), dS^T = P^T (dP^T - Delta)   (CUDA cores)
-//        dV  += P^T dO       (A from TMEM)     dK  += dS^T Q     (TMEM)
-//        dQ_i = dS K         (TMEM) -> added into a float32 accumulator.
-//      dK, dV leave through a TMA store at the end.
-//   3. s2_bwd_dq_convert: dq = bf16(scale · accumulator).
-// Warp roles of s2_bwd_kernel (320 threads): warps 0-7 elementwise work, the
-// two warpgroups splitting the 128 query columns in halves (thread = one key
-// row = one TMEM lane); warp 8 TMA producer; warp 9 TMEM allocator and MMA
-// issuer.  TMEM (512 columns): S^T / P^T [0,128), dP^T / dQ [128,256),
-// dV [256, 256+D), dK [256+D, 256+2D).
+//   2. s2_bwd_dkdv_kernel: key-major, one CTA per 128-key tile of a segment,
+//      walking the query tiles from the diagonal to the segment's end:
+//        S^T = K Q^T, dP^T = V dO^T (TMEM);  P^T = exp2(S^T·c - lse2) and
+//        dS^T = P^T (dP^T - Delta) on the CUDA cores, both written back to
+//        TMEM as bf16;  dV += P^T dO and dK += dS^T Q with A read from TMEM.
+//   3. s2_bwd_dq_kernel: query-major, one CTA per 128-query tile, walking the
+//      key tiles from the segment start to the diagonal:
+//        S = Q K^T, dP = dO V^T (TMEM);  dS = P (dP - Delta) -> TMEM (bf16);
+//        dQ += dS K with A read from TMEM;  dq = bf16(dQ / sqrt(D)).
+// The dq pass recomputes S and dP (two of its three products), so the
+// backward does 7 instead of 5 tile products per (key tile, query tile) pair.
+// In exchange dq is written once, in bf16, without a float32 accumulator:
+// a fused kernel adds one float32 partial of every dq row per key tile into
+// global memory, and the L2's float32 reduction rate (a few TB/s) then bounds
+// the whole backward.  dq is also bitwise deterministic this way.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -36,50 +38,65 @@ namespace s2 {
 
 namespace bwd {
 
-constexpr int kThreads = 320;
-constexpr int kStages = 2;
-constexpr int kChunkBytes = kTile * 64 * 2;
+constexpr int kThreads = 320;  // warps 0-7 elementwise, 8 TMA producer, 9 TMEM + MMA issuer
+constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16: one 128-byte-swizzle column block
 
-enum Bar {
-  KV_FULL = 0,
-  QD_FULL = 1,   // + stage (2)
-  QD_EMPTY = 3,  // + stage (2)
-  S_FULL = 5,
-  DP_FULL = 6,
-  DS_READY = 7,
-  DV_DONE = 8,
-  DQ_FULL = 9,
-  DQ_FREE = 10,
-  ACC_DONE = 11,
-  S_READ = 12,   // both elementwise warpgroups have read S^T (before P^T overwrites it)
-  NUM_BARS = 13
-};
+// Descriptor offsets (16-byte units) of MMA K-step kk over a 128-byte-swizzled
+// tile: K-major operands step 32 bytes inside a 64-column chunk, then a chunk;
+// MN-major operands step 16 rows.
+#define S2_KM_OFF(kk) ((uint64_t)((((kk) / 4) * kChunkBytes + ((kk) % 4) * 32) >> 4))
+#define S2_MN_OFF(kk) ((uint64_t)(((kk) * 2048) >> 4))
 
-template <int D>
-struct Layout {
-  static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kK = 0;
-  static constexpr int kV = kTileBytes;
-  static constexpr int kQ = 2 * kTileBytes;                    // + stage * kTileBytes
-  static constexpr int kdO = kQ + kStages * kTileBytes;        // + stage * kTileBytes
-  static constexpr int kdS = kdO + kStages * kTileBytes;       // 128 x 128 bf16
-  static constexpr int kBars = kdS + kTile * kTile * 2;
-  static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
-  static constexpr int kAlloc = kBytes + 1024;
-};
-
+// Next query tile after qt (up to the segment end) that holds a valid row, or -1.
 __device__ __forceinline__ int next_q(const Plan& p, const Unit& u, int qt) {
   for (int j = qt + 1; j <= u.kmax; ++j)
     if (ktile_valid(p, u, j)) return j;
   return -1;
 }
 
+// Next valid key tile after k (up to the query tile u.t[0]), or -1.
+__device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k) {
+  for (int j = k + 1; j <= u.t[0]; ++j)
+    if (ktile_valid(p, u, j)) return j;
+  return -1;
+}
+
+// An accumulator (TMEM, lane = row) -> bf16 -> shared staging laid out as
+// two 128-byte-swizzled chunks of 64 columns; warpgroup x converts columns
+// [x·D/2, x·D/2 + D/2) of its row.  Rows that are not valid are written as 0.
+template <int D>
+__device__ __forceinline__ void acc_to_smem(uint32_t tacc, uint32_t lane_off, int x, int row, bool have,
+                                            bool row_valid, float mul, uint32_t stage) {
+#pragma unroll
+  for (int c2 = 0; c2 < D / 64; ++c2) {
+    const int d0 = x * (D / 2) + 32 * c2;
+    uint32_t v[32];
+    if (have) {
+      tmem_ld32(tacc + lane_off + d0, v);
+      tmem_wait_ld();
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int col = d0 + 8 * q;
+      const int chunk = col / 64, piece = (col % 64) / 8;
+      uint32_t w[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float a = (have && row_valid) ? __uint_as_float(v[8 * q + 2 * t]) * mul : 0.f;
+        const float b = (have && row_valid) ? __uint_as_float(v[8 * q + 2 * t + 1]) * mul : 0.f;
+        w[t] = pack_bf16(a, b);
+      }
+      st_shared_v4(stage + chunk * kChunkBytes + row * 128 + ((piece ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 }  // namespace bwd
 
 // ------------------------------------------------------------------ preprocess
 // kTpr = D/8 threads per (b, i, h) row, 8 bf16 (16 bytes) each.  Stores the
-// negated statistics the main kernel adds: -Delta = -(dout·o) and
-// -lse·log2(e) (-inf on padded rows, which zeroes their probabilities).
+// negated statistics the passes add: -Delta = -(dout·o) and -lse·log2(e)
+// (-inf on padded rows, which zeroes their probabilities).
 template <int D>
 __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restrict__ o,
                                                    const __nv_bfloat16* __restrict__ dout,
@@ -116,384 +133,66 @@ __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restric
   }
 }
 
-// ------------------------------------------------------------------ dq convert
-__global__ void __launch_bounds__(256) s2_bwd_dq_convert(const float4* __restrict__ acc,
-                                                          uint2* __restrict__ dq, long long n4, float scale) {
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
-    const float4 a = acc[i];
-    uint2 r;
-    r.x = pack_bf16(a.x * scale, a.y * scale);
-    r.y = pack_bf16(a.z * scale, a.w * scale);
-    dq[i] = r;
-  }
-}
+// ------------------------------------------------------------------ dK, dV pass
+// Tensor memory (512 columns): R1 [0, 128) S^T then P^T; R2 [128, 256) dP^T
+// then dS^T; dV [256, 256 + D); dK [256 + D, 256 + 2D).  P^T and dS^T are
+// bf16 pairs: query columns [64x, 64x + 64) of a tile land in columns
+// [64x, 64x + 32) of their region, which warpgroup x has already read.
+// Issue order per query tile n (one thread of warp 9):
+//   dP(n) -> R2    (behind dK(n-1), the last reader of dS^T(n-1))
+//   dV(n)          once P^T(n) is in R1
+//   S(n+1) -> R1   (behind dV(n), the last reader of P^T(n))
+//   dK(n)          once dS^T(n) is in R2
+// so the exponentials of tile n+1 overlap dK(n) and dP(n+1), and dS(n)
+// overlaps dV(n) and S(n+1).  Elementwise thread = key row j (TMEM lane),
+// warpgroup x = query columns [64x, 64x + 64); order P(0), [dS(n), P(n+1)].
+namespace dkdv {
 
-// ------------------------------------------------------------------ main backward kernel
-template <int D>
-__global__ void __launch_bounds__(bwd::kThreads, 1)
-    s2_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                  const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                  const Plan p, const float* __restrict__ delta, const float* __restrict__ lse2,
-                  float* __restrict__ dq_acc, int* __restrict__ status) {
-  using namespace bwd;
-  using L = Layout<D>;
-  constexpr int kChunks = D / 64;
-
-  Unit u;
-  if (!decode_kv_unit(p, blockIdx.x, u)) return;
-  const int kt = u.t[0];
-  const int k0 = tile_orig(p, u, kt);
-  const bool kvalid = u.part[0];
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto bar = [&](int i) { return smem_u32(&bars[i]); };
-  const uint32_t sK = sb + L::kK, sV = sb + L::kV, sdS = sb + L::kdS;
-  auto sQ = [&](int st) { return sb + L::kQ + st * L::kTileBytes; };
-  auto sdO = [&](int st) { return sb + L::kdO + st * L::kTileBytes; };
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) {
-    mbar_init(bar(KV_FULL), 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(bar(QD_FULL + s), 1);
-      mbar_init(bar(QD_EMPTY + s), 1);
-    }
-    mbar_init(bar(S_FULL), 1);
-    mbar_init(bar(DP_FULL), 1);
-    mbar_init(bar(DS_READY), 256);
-    mbar_init(bar(DV_DONE), 1);
-    mbar_init(bar(DQ_FULL), 1);
-    mbar_init(bar(DQ_FREE), 256);
-    mbar_init(bar(ACC_DONE), 1);
-    mbar_init(bar(S_READ), 256);
-    *abort_flag = 0;
-    fence_barrier_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == 9) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
-  const int row_base = u.b * p.N;
-
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && kvalid) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmdO);
-      mbar_arrive_expect_tx(bar(KV_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < kChunks; ++c) {
-        tma_load_3d(sK + c * kChunkBytes, &tmK, c * 64, u.h, row_base + k0, bar(KV_FULL));
-        tma_load_3d(sV + c * kChunkBytes, &tmV, c * 64, u.h, row_base + k0, bar(KV_FULL));
-      }
-      int n = 0;
-      bool ok = true;
-      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt)) {
-        if (qt == kt && !ktile_valid(p, u, qt)) continue;
-        const int st = n % kStages;
-        if (n >= kStages) ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(QD_FULL + st), 2 * L::kTileBytes);
-        const int q0 = tile_orig(p, u, qt);
-        for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(sQ(st) + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
-          tma_load_3d(sdO(st) + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
-        }
-        ++n;
-      }
-      for (int d = (n > kStages ? n - kStages : 0); d < n; ++d)
-        s2_wait(bar(QD_FULL + d % kStages), (d / kStages) & 1, abort_flag, status, 8);
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && kvalid) {
-      constexpr uint32_t id_st = umma_idesc_bf16(128, 128, 0, 0);  // S^T, dP^T: K-major A and B
-      constexpr uint32_t id_dv = umma_idesc_bf16(128, D, 0, 1);    // dV: A in TMEM, B = dO MN-major
-      constexpr uint32_t id_dk = umma_idesc_bf16(128, D, 0, 1);    // dK: A = dS^T K-major, B = Q MN-major
-      constexpr uint32_t id_dq = umma_idesc_bf16(128, D, 1, 1);    // dQ: A = dS MN-major, B = K MN-major
-      bool ok = s2_wait(bar(KV_FULL), 0, abort_flag, status, 16);
-      tc_fence_after();
-      int n = 0;
-      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt)) {
-        if (qt == kt && !ktile_valid(p, u, qt)) continue;
-        const int st = n % kStages;
-        ok = s2_wait(bar(QD_FULL + st), (n / kStages) & 1, abort_flag, status, 16);
-        if (!ok) break;
-        tc_fence_after();
-        if (n > 0) {  // P^T(n-1) in the S columns must have been consumed by dV(n-1)
-          ok = s2_wait(bar(DV_DONE), (n - 1) & 1, abort_flag, status, 16);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-          umma_ss(tS, umma_desc_sw128(sK + off, 16, 1024), umma_desc_sw128(sQ(st) + off, 16, 1024), id_st, kk > 0);
-        }
-        umma_commit(bar(S_FULL));
-        if (n > 0) {  // dQ(n-1) in the dP columns must have been read out
-          ok = s2_wait(bar(DQ_FREE), (n - 1) & 1, abort_flag, status, 16);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-          umma_ss(tDP, umma_desc_sw128(sV + off, 16, 1024), umma_desc_sw128(sdO(st) + off, 16, 1024), id_st, kk > 0);
-        }
-        umma_commit(bar(DP_FULL));
-        ok = s2_wait(bar(DS_READY), n & 1, abort_flag, status, 16);
-        if (!ok) break;
-        tc_fence_after();
-        // dV += P^T dO : K = 128 queries, A = P^T packed two per TMEM column
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tdV, tS + kk * 8, umma_desc_sw128(sdO(st) + kk * 2048, kChunkBytes, 1024), id_dv,
-                  (n > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(DV_DONE));
-        // dK += dS^T Q
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          const uint32_t aoff = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-          umma_ss(tdK, umma_desc_sw128(sdS + aoff, 16, 1024),
-                  umma_desc_sw128(sQ(st) + kk * 2048, kChunkBytes, 1024), id_dk, (n > 0 || kk > 0) ? 1u : 0u);
-        }
-        // dQ = dS K : M = 128 queries, K = 128 keys; both operands MN-major
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ss(tDP, umma_desc_sw128(sdS + kk * 2048, kChunkBytes, 1024),
-                  umma_desc_sw128(sK + kk * 2048, kChunkBytes, 1024), id_dq, kk > 0 ? 1u : 0u);
-        umma_commit(bar(DQ_FULL));
-        umma_commit(bar(QD_EMPTY + st));
-        ++n;
-      }
-      umma_commit(bar(ACC_DONE));
-      s2_wait(bar(ACC_DONE), 0, abort_flag, status, 16);
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ elementwise warpgroups
-    const int x = warp / 4;            // column half: queries [64x, 64x + 64)
-    const int j = (warp % 4) * 32 + lane;  // key row == TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
-    const size_t stat_base = ((size_t)u.b * p.H + u.h) * p.N;
-    bool ok = true;
-    int n = 0;
-    if (kvalid) {
-      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt)) {
-        if (qt == kt && !ktile_valid(p, u, qt)) continue;
-        const int q0 = tile_orig(p, u, qt);
-        int lo, hi;
-        query_range(p, u, kt, qt, j, lo, hi);
-        ok = s2_wait(bar(S_FULL), n & 1, abort_flag, status, 32);
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t sv[64];
-        tmem_ld32(tS + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_wait_ld();
-        // both halves must have read S^T before either overwrites it with P^T
-        mbar_arrive(bar(S_READ));
-        ok = s2_wait(bar(S_READ), n & 1, abort_flag, status, 32);
-        if (!ok) break;
-        ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int col0 = 64 * x + 32 * c;
-          uint32_t dp[32];
-          tmem_ld32(tDP + lane_off + col0, dp);
-          tmem_wait_ld();
-          const float4* l4 = reinterpret_cast<const float4*>(lse2 + stat_base + q0 + col0);
-          const float4* d4 = reinterpret_cast<const float4*>(delta + stat_base + q0 + col0);
-          uint32_t pp[16], dsp[16];
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const float4 lv = __ldg(l4 + g), dv = __ldg(d4 + g);
-            const float lsv[4] = {lv.x, lv.y, lv.z, lv.w};
-            const float dlv[4] = {dv.x, dv.y, dv.z, dv.w};
-            float pv[4], dsv[4];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const int i = 4 * g + t;
-              const int col = col0 + i;
-              const bool vis = (col >= lo) && (col < hi);
-              const float pr = vis ? ex2(fmaf(__uint_as_float(sv[32 * c + i]), p.scale_log2, lsv[t])) : 0.f;
-              pv[t] = pr;
-              dsv[t] = pr * (__uint_as_float(dp[i]) + dlv[t]);
-            }
-            pp[2 * g] = pack_bf16(pv[0], pv[1]);
-            pp[2 * g + 1] = pack_bf16(pv[2], pv[3]);
-            dsp[2 * g] = pack_bf16(dsv[0], dsv[1]);
-            dsp[2 * g + 1] = pack_bf16(dsv[2], dsv[3]);
-          }
-          tmem_st16(tS + lane_off + col0 / 2, pp);
-          // dS^T row j, columns col0..col0+31: chunk x, 16-byte pieces 4c..4c+3
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int piece = 4 * c + q;
-            const uint32_t addr = sdS + x * kChunkBytes + j * 128 + ((piece ^ (j & 7)) << 4);
-            st_shared_v4(addr, dsp[4 * q], dsp[4 * q + 1], dsp[4 * q + 2], dsp[4 * q + 3]);
-          }
-        }
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(bar(DS_READY));
-        // dQ tile (thread = query row j of this query tile): add into the accumulator
-        ok = s2_wait(bar(DQ_FULL), n & 1, abort_flag, status, 32);
-        if (!ok) break;
-        tc_fence_after();
-        const bool qrow_valid = q0 + j < p.n_valid;
-#pragma unroll
-        for (int c2 = 0; c2 < D / 64; ++c2) {
-          const int d0 = x * (D / 2) + 32 * c2;
-          uint32_t dq[32];
-          tmem_ld32(tDP + lane_off + d0, dq);
-          tmem_wait_ld();
-          if (qrow_valid) {
-            float* dst = dq_acc + (((size_t)row_base + q0 + j) * p.H + u.h) * D + d0;
-#pragma unroll
-            for (int g = 0; g < 8; ++g)
-              red_add_v4(dst + 4 * g, __uint_as_float(dq[4 * g]), __uint_as_float(dq[4 * g + 1]),
-                         __uint_as_float(dq[4 * g + 2]), __uint_as_float(dq[4 * g + 3]));
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar(DQ_FREE));
-        ++n;
-      }
-    }
-    // ---------------------------------------------------------- epilogue: dK, dV
-    bool have = kvalid && ok && n > 0;
-    if (have) {
-      have = s2_wait(bar(ACC_DONE), 0, abort_flag, status, 32);
-      tc_fence_after();
-    }
-    const bool key_valid = have && (k0 + j < p.n_valid);
-    const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
-    // staging: dV -> Q stage 0, dK -> Q stage 1 (free once every MMA has completed)
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t tsrc = which == 0 ? tdV : tdK;
-      const float mul = which == 0 ? 1.f : scale;
-      const uint32_t stage = sQ(which);
-#pragma unroll
-      for (int c2 = 0; c2 < D / 64; ++c2) {
-        const int d0 = x * (D / 2) + 32 * c2;
-        uint32_t v[32];
-        if (have) {
-          tmem_ld32(tsrc + lane_off + d0, v);
-          tmem_wait_ld();
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = d0 + 8 * q;
-          const int chunk = col / 64, piece = (col % 64) / 8;
-          uint32_t w[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float a = key_valid ? __uint_as_float(v[8 * q + 2 * t]) * mul : 0.f;
-            const float b = key_valid ? __uint_as_float(v[8 * q + 2 * t + 1]) * mul : 0.f;
-            w[t] = pack_bf16(a, b);
-          }
-          st_shared_v4(stage + chunk * kChunkBytes + j * 128 + ((piece ^ (j & 7)) << 4), w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
-    fence_proxy_async_smem();
-    named_bar_sync(2, 256);
-    if (threadIdx.x == 0) {
-      for (int c = 0; c < kChunks; ++c) {
-        tma_store_3d(&tmdV, sQ(0) + c * kChunkBytes, c * 64, u.h, row_base + k0);
-        tma_store_3d(&tmdK, sQ(1) + c * kChunkBytes, c * 64, u.h, row_base + k0);
-      }
-      tma_store_commit();
-      tma_store_wait_all();
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
-// ------------------------------------------------------------------ split backward kernel (D = 128)
-// Same CTA decomposition (one 128-key tile, query tiles from the diagonal to
-// the segment end), but every query tile is processed as two 64-query halves,
-// half x by warpgroup x, so that one half's elementwise work runs while the
-// tensor core works on the other half:
-//   S^T_x  = K Q_x^T          (M 128 keys, N 64 queries)   TMEM [64x, 64x+64)
-//   dP^T_x = V dO_x^T                                        TMEM [128+64x, ...)
-//   P^T_x (bf16, into the dP^T_x columns), dS^T_x (bf16, shared memory)
-//   dV += P^T_x dO_x (A from TMEM),  dK += dS^T_x Q_x
-//   dQ^T_x = K^T dS^T_x       (M = D = 128, N 64 queries) -> the S^T_x columns
-// dQ^T puts d on the TMEM lanes, so each warp's float32 atomic adds into the
-// dq accumulator cover 128 contiguous bytes of one query row.
-namespace bwds {
-
-constexpr int D = 128;
-constexpr int kThreads = 320;
 constexpr int kStages = 2;
-constexpr int kChunkBytes = kTile * 64 * 2;
-
 enum Bar {
   KV_FULL = 0,
-  QD_FULL = 1,    // + stage (2)
-  QD_EMPTY = 3,   // + stage (2)
-  SP_FULL = 5,    // + half (2)
-  DS_READY = 7,   // + half (2)
-  DQ_FULL = 9,    // + half (2)
-  DQ_FREE = 11,   // + half (2)
-  ACC_DONE = 13,
-  RED_DONE = 14,  // + stage (2): both halves' dQ reductions have read their staging rows
-  NUM_BARS = 16
+  QD_FULL = 1,   // + stage (2)
+  QD_EMPTY = 3,  // + stage (2)
+  S_FULL = 5,
+  DP_FULL = 6,
+  P_READY = 7,
+  DS_READY = 8,
+  ACC_DONE = 9,
+  NUM_BARS = 10
 };
 
+template <int D>
 struct Layout {
-  static constexpr int kTileBytes = kTile * D * 2;       // 32 KB
-  static constexpr int kHalfBytes = kTile * 64 * 2;      // 16 KB: dS^T of one half
-  static constexpr int kStatBytes = 2 * kTile * 4;       // lse2[128], delta[128]
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kStatBytes = 2 * kTile * 4;  // -lse2[128], -Delta[128] of a query tile
   static constexpr int kK = 0;
   static constexpr int kV = kTileBytes;
-  static constexpr int kQ = 2 * kTileBytes;
-  static constexpr int kdO = kQ + kStages * kTileBytes;
-  static constexpr int kdS = kdO + kStages * kTileBytes;
-  static constexpr int kStat = kdS + 2 * kHalfBytes;
+  static constexpr int kQ = 2 * kTileBytes;               // + stage * kTileBytes
+  static constexpr int kdO = kQ + kStages * kTileBytes;   // + stage * kTileBytes
+  static constexpr int kStat = kdO + kStages * kTileBytes;  // + stage * kStatBytes
   static constexpr int kBars = kStat + kStages * kStatBytes;
   static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
 };
 
-}  // namespace bwds
+}  // namespace dkdv
 
-__global__ void __launch_bounds__(bwds::kThreads, 1)
-    s2_bwd_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                        const __grid_constant__ CUtensorMap tmdQacc, const Plan p, const float* __restrict__ delta,
-                        const float* __restrict__ lse2, int* __restrict__ status) {
-  using namespace bwds;
-  using L = bwds::Layout;
+template <int D>
+__global__ void __launch_bounds__(bwd::kThreads, 1)
+    s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                       const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                       const Plan p, const float* __restrict__ delta, const float* __restrict__ lse2,
+                       int* __restrict__ status) {
+  using namespace bwd;
+  using namespace dkdv;
+  using L = dkdv::Layout<D>;
   constexpr int kChunks = D / 64;
 
   Unit u;
   if (!decode_kv_unit(p, blockIdx.x, u)) return;
-  extern __shared__ __align__(1024) uint8_t smem_split[];
-  // The layout needs a 1024-byte aligned base (128-byte swizzle atoms); the
-  // dynamic window starts aligned in practice.  If it ever does not, report
-  // and leave instead of computing on misaligned tiles.
-  if (smem_u32(smem_split) & 1023u) {
+  extern __shared__ __align__(1024) uint8_t smem_kv[];
+  // 128-byte swizzle atoms need a 1024-byte aligned base; report and leave otherwise.
+  if (smem_u32(smem_kv) & 1023u) {
     if (threadIdx.x == 0) atomicOr(status, 256);
     return;
   }
@@ -501,30 +200,27 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
   const int k0 = tile_orig(p, u, kt);
   const bool kvalid = u.part[0];
 
-  uint8_t* smem = smem_split;
+  uint8_t* smem = smem_kv;
   const uint32_t sb = smem_u32(smem);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  const uint32_t sbar = sb + L::kBars;
+#define bar(i) (sbar + 8u * (uint32_t)(i))
+#define sQ(st) (sb + L::kQ + (uint32_t)(st) * L::kTileBytes)
+#define sdO(st) (sb + L::kdO + (uint32_t)(st) * L::kTileBytes)
   const uint32_t sK = sb + L::kK, sV = sb + L::kV;
-  auto sQ = [&](int st) { return sb + L::kQ + st * L::kTileBytes; };
-  auto sdO = [&](int st) { return sb + L::kdO + st * L::kTileBytes; };
-  auto sdS = [&](int x) { return sb + L::kdS + x * L::kHalfBytes; };
-  auto sStat = [&](int st) { return sb + L::kStat + st * L::kStatBytes; };
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     mbar_init(bar(KV_FULL), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(bar(QD_FULL + i), 1);
       mbar_init(bar(QD_EMPTY + i), 1);
-      mbar_init(bar(SP_FULL + i), 1);
-      mbar_init(bar(DS_READY + i), 128);
-      mbar_init(bar(DQ_FULL + i), 1);
-      mbar_init(bar(DQ_FREE + i), 128);
-      mbar_init(bar(RED_DONE + i), 2);
     }
+    mbar_init(bar(S_FULL), 1);
+    mbar_init(bar(DP_FULL), 1);
+    mbar_init(bar(P_READY), 256);
+    mbar_init(bar(DS_READY), 256);
     mbar_init(bar(ACC_DONE), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -538,9 +234,7 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto tS = [&](int x) { return tmem + 64 * x; };
-  auto tDP = [&](int x) { return tmem + 128 + 64 * x; };
-  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
+  const uint32_t tR1 = tmem, tR2 = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
   const int row_base = u.b * p.N;
   const size_t stat_base = ((size_t)u.b * p.H + u.h) * p.N;
 
@@ -556,12 +250,9 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
       }
       int n = 0;
       bool ok = true;
-      for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
+      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt)) {
         const int st = n % kStages;
-        if (n >= kStages) {  // MMAs done with the stage, and the dQ reductions staged in it have read it
-          ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
-          if (ok) ok = s2_wait(bar(RED_DONE + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
-        }
+        if (n >= kStages) ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(QD_FULL + st), 2 * L::kTileBytes + L::kStatBytes);
         const int q0 = tile_orig(p, u, qt);
@@ -569,10 +260,12 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
           tma_load_3d(sQ(st) + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
           tma_load_3d(sdO(st) + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
         }
-        bulk_load(sStat(st), lse2 + stat_base + q0, kTile * 4, bar(QD_FULL + st));
-        bulk_load(sStat(st) + kTile * 4, delta + stat_base + q0, kTile * 4, bar(QD_FULL + st));
+        const uint32_t sstat = sb + L::kStat + st * L::kStatBytes;
+        bulk_load(sstat, lse2 + stat_base + q0, kTile * 4, bar(QD_FULL + st));
+        bulk_load(sstat + kTile * 4, delta + stat_base + q0, kTile * 4, bar(QD_FULL + st));
         ++n;
       }
+      // the last loads must land before the CTA retires
       for (int d = (n > kStages ? n - kStages : 0); d < n; ++d)
         s2_wait(bar(QD_FULL + d % kStages), (d / kStages) & 1, abort_flag, status, 8);
     }
@@ -580,101 +273,101 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
   } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && kvalid) {
-      constexpr uint32_t id_sp = umma_idesc_bf16(128, 64, 0, 0);   // S^T_x, dP^T_x
-      constexpr uint32_t id_acc = umma_idesc_bf16(128, D, 0, 1);   // dV (A in TMEM), dK
-      constexpr uint32_t id_dq = umma_idesc_bf16(128, 64, 1, 1);   // dQ^T_x = K^T dS^T_x
+      constexpr uint32_t id_s = umma_idesc_bf16(128, 128, 0, 0);  // S^T, dP^T: M keys, N queries, K-major
+      constexpr uint32_t id_acc = umma_idesc_bf16(128, D, 0, 1);  // dV, dK: A from TMEM, B MN-major
+      // Descriptors are built once; each MMA adds a compile-time offset.
+      const uint64_t dK_km = umma_desc_sw128(sK, 16, 1024), dV_km = umma_desc_sw128(sV, 16, 1024);
+      const uint64_t dQ_km = umma_desc_sw128(sQ(0), 16, 1024), ddO_km = umma_desc_sw128(sdO(0), 16, 1024);
+      const uint64_t dQ_mn = umma_desc_sw128(sQ(0), kChunkBytes, 1024);
+      const uint64_t ddO_mn = umma_desc_sw128(sdO(0), kChunkBytes, 1024);
+      constexpr uint64_t kStageStep = (uint64_t)(L::kTileBytes >> 4);
       bool ok = s2_wait(bar(KV_FULL), 0, abort_flag, status, 16);
+      if (ok) ok = s2_wait(bar(QD_FULL + 0), 0, abort_flag, status, 16);
       tc_fence_after();
+      if (ok) {  // S(0)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) umma_ss(tR1, dK_km + S2_KM_OFF(kk), dQ_km + S2_KM_OFF(kk), id_s, kk > 0);
+        umma_commit(bar(S_FULL));
+      }
       int n = 0;
-      for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
+      for (int qt = kt; ok && qt >= 0;) {
         const int st = n % kStages;
-        ok = s2_wait(bar(QD_FULL + st), (n / kStages) & 1, abort_flag, status, 16);
+        const uint64_t so = (uint64_t)st * kStageStep;
+        const int qn = next_q(p, u, qt);
+        // dP^T(n) -> R2
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tR2, dV_km + S2_KM_OFF(kk), ddO_km + so + S2_KM_OFF(kk), id_s, kk > 0);
+        umma_commit(bar(DP_FULL));
+        // dV += P^T(n) dO(n): K = 128 queries, 16 per step, P^T pairs at R1 + 64·(kk/4) + 8·(kk%4)
+        ok = s2_wait(bar(P_READY), n & 1, abort_flag, status, 16);
         if (!ok) break;
         tc_fence_after();
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (n > 0) {  // dQ^T_x(n-1) read out of the S columns, P^T_x(n-1) consumed
-            ok = s2_wait(bar(DQ_FREE + x), (n - 1) & 1, abort_flag, status, 16);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          const uint32_t qrow = x * 64 * 128;  // first query row of the half inside a 64-column chunk
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-            umma_ss(tS(x), umma_desc_sw128(sK + off, 16, 1024), umma_desc_sw128(sQ(st) + off + qrow, 16, 1024),
-                    id_sp, kk > 0);
-          }
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * kChunkBytes + (kk % 4) * 32;
-            umma_ss(tDP(x), umma_desc_sw128(sV + off, 16, 1024), umma_desc_sw128(sdO(st) + off + qrow, 16, 1024),
-                    id_sp, kk > 0);
-          }
-          umma_commit(bar(SP_FULL + x));
-        }
-        for (int x = 0; x < 2 && ok; ++x) {
-          ok = s2_wait(bar(DS_READY + x), n & 1, abort_flag, status, 16);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tdV, tR1 + 64 * (kk / 4) + 8 * (kk % 4), ddO_mn + so + S2_MN_OFF(kk), id_acc,
+                  (n > 0 || kk > 0) ? 1u : 0u);
+        // S^T(n+1) -> R1
+        if (qn >= 0) {
+          const int st1 = (n + 1) % kStages;
+          ok = s2_wait(bar(QD_FULL + st1), ((n + 1) / kStages) & 1, abort_flag, status, 16);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t qrow = x * 64 * 128;
-          const bool first = (n == 0 && x == 0);
-          // dV += P^T_x dO_x : K = 64 queries of the half
-          for (int kk = 0; kk < 4; ++kk)
-            umma_ts(tdV, tDP(x) + kk * 8, umma_desc_sw128(sdO(st) + qrow + kk * 2048, kChunkBytes, 1024), id_acc,
-                    (!first || kk > 0) ? 1u : 0u);
-          // dK += dS^T_x Q_x
-          for (int kk = 0; kk < 4; ++kk)
-            umma_ss(tdK, umma_desc_sw128(sdS(x) + kk * 32, 16, 1024),
-                    umma_desc_sw128(sQ(st) + qrow + kk * 2048, kChunkBytes, 1024), id_acc,
-                    (!first || kk > 0) ? 1u : 0u);
-          // dQ^T_x = K^T dS^T_x : M = D, K = 128 keys
-          for (int kk = 0; kk < kTile / 16; ++kk)
-            umma_ss(tS(x), umma_desc_sw128(sK + kk * 2048, kChunkBytes, 1024),
-                    umma_desc_sw128(sdS(x) + kk * 2048, kChunkBytes, 1024), id_dq, kk > 0 ? 1u : 0u);
-          umma_commit(bar(DQ_FULL + x));
+          const uint64_t so1 = (uint64_t)st1 * kStageStep;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ss(tR1, dK_km + S2_KM_OFF(kk), dQ_km + so1 + S2_KM_OFF(kk), id_s, kk > 0);
+          umma_commit(bar(S_FULL));
         }
+        // dK += dS^T(n) Q(n), dS^T pairs at R2 + 64·(kk/4) + 8·(kk%4)
+        ok = s2_wait(bar(DS_READY), n & 1, abort_flag, status, 16);
         if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tdK, tR2 + 64 * (kk / 4) + 8 * (kk % 4), dQ_mn + so + S2_MN_OFF(kk), id_acc,
+                  (n > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(QD_EMPTY + st));
         ++n;
+        qt = qn;
       }
+      // every issued MMA must be complete before TMEM is read or released
       umma_commit(bar(ACC_DONE));
       s2_wait(bar(ACC_DONE), 0, abort_flag, status, 16);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise warpgroups
-    const int x = warp / 4;                 // query half [64x, 64x + 64)
-    const int j = (warp % 4) * 32 + lane;   // key row == TMEM lane (also d for dQ^T)
+    const int x = warp / 4;                // query columns [64x, 64x + 64)
+    const int j = (warp % 4) * 32 + lane;  // key row == TMEM lane
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
     bool ok = true;
     int n = 0;
     if (kvalid) {
       const bool key_tile_ragged = k0 + kTile > p.n_valid;
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
-      for (int qt = kt; ok && qt >= 0; qt = bwd::next_q(p, u, qt)) {
-        const int st = n % kStages;
-        const int q0 = tile_orig(p, u, qt);
-        // masks are needed on the diagonal tile and on a key tile with padding;
-        // padded queries are zeroed by their -inf statistic
-        const bool masked = (qt == kt) || key_tile_ragged;
+      float pf[64];  // P of the current tile (fp32), from its exponentials to its dS
+      // P(nn): S^T -> P^T (bf16 pairs into R1) and pf
+      auto p_step = [&](int nn, int qtile) -> bool {
+        const int st = nn % kStages;
+        // masks on the diagonal tile and on a key tile with padding; padded
+        // queries are zeroed by their -inf statistic
+        const bool masked = (qtile == kt) || key_tile_ragged;
         int lo = 0, hi = kTile;
-        if (masked) query_range(p, u, kt, qt, j, lo, hi);
-        // the stage's -lse2 / -Delta rows come with its Q/dO tiles
-        ok = s2_wait(bar(QD_FULL + st), (n / kStages) & 1, abort_flag, status, 32);
-        if (!ok) break;
-        ok = s2_wait(bar(SP_FULL + x), n & 1, abort_flag, status, 32);
-        if (!ok) break;
+        if (masked) query_range(p, u, kt, qtile, j, lo, hi);
+        if (!s2_wait(bar(QD_FULL + st), (nn / kStages) & 1, abort_flag, status, 32)) return false;
+        if (!s2_wait(bar(S_FULL), nn & 1, abort_flag, status, 32)) return false;
         tc_fence_after();
         const float2* nl = reinterpret_cast<const float2*>(smem + L::kStat + st * L::kStatBytes) + 32 * x;
-        const float2* nd = nl + kTile / 2;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {  // 32 query columns per chunk
-          uint32_t sv[32], dp[32];
-          tmem_ld32(tS(x) + lane_off + 32 * c, sv);
-          tmem_ld32(tDP(x) + lane_off + 32 * c, dp);
+        for (int c = 0; c < 2; ++c) {  // 32 query columns at a time
+          uint32_t sv[32];
+          tmem_ld32(tR1 + lane_off + 64 * x + 32 * c, sv);
           tmem_wait_ld();
-          uint32_t pp[16], dsp[16];
+          uint32_t pp[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            // P = 2^(S·log2(e)/sqrt(D) - lse·log2(e)),  dS = P (dP - Delta), two columns at a time
+            // P = 2^(S·log2(e)/sqrt(D) - lse·log2(e)), two columns at a time
             const float2 a =
                 __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl[16 * c + i]);
             float p0 = ex2(a.x), p1 = ex2(a.y);
@@ -683,102 +376,64 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
               p0 = (col >= lo && col < hi) ? p0 : 0.f;
               p1 = (col + 1 >= lo && col + 1 < hi) ? p1 : 0.f;
             }
-            const float2 d2 =
-                __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[16 * c + i]);
-            const float2 ds = __fmul2_rn(make_float2(p0, p1), d2);
+            pf[32 * c + 2 * i] = p0;
+            pf[32 * c + 2 * i + 1] = p1;
             pp[i] = pack_bf16(p0, p1);
-            dsp[i] = pack_bf16(ds.x, ds.y);
           }
-          // P^T (bf16 pairs) into dP^T_x columns [16c, 16c + 16), already read
-          tmem_st16(tDP(x) + lane_off + 16 * c, pp);
-          // dS^T row j, queries [32c, 32c + 32): 16-byte pieces 4c..4c+3, 128-byte swizzle
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int piece = 4 * c + q;
-            st_shared_v4(sdS(x) + j * 128 + ((piece ^ (j & 7)) << 4), dsp[4 * q], dsp[4 * q + 1], dsp[4 * q + 2],
-                         dsp[4 * q + 3]);
-          }
+          tmem_st16(tR1 + lane_off + 64 * x + 16 * c, pp);
         }
         tmem_wait_st();
-        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(DS_READY + x));
-        // dQ^T_x (lane = d, columns = the half's 64 queries): into registers, then
-        // release the TMEM columns at once so the next S^T_x / dP^T_x can start
-        ok = s2_wait(bar(DQ_FULL + x), n & 1, abort_flag, status, 32);
+        mbar_arrive(bar(P_READY));
+        return true;
+      };
+      int qt = kt;
+      ok = p_step(0, qt);
+      while (ok && qt >= 0) {
+        const int st = n % kStages;
+        const int qn = next_q(p, u, qt);
+        // dS(n) = P (dP - Delta) -> dS^T pairs into R2
+        ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
         if (!ok) break;
         tc_fence_after();
-        uint32_t dq[64];
-        tmem_ld32(tS(x) + lane_off, *reinterpret_cast<uint32_t(*)[32]>(&dq[0]));
-        tmem_ld32(tS(x) + lane_off + 32, *reinterpret_cast<uint32_t(*)[32]>(&dq[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(DQ_FREE + x));
-        // Add into the fp32 accumulator with bulk tensor reductions, staged in this
-        // half's rows [64x, 64x + 64) of the stage's Q and dO tiles: every MMA
-        // reading them (S^T_x, dP^T_x, dV_x, dK_x) has completed at DQ_FULL[x], the
-        // other half never reads them, and the producer refills the stage only
-        // after RED_DONE.  Four 8 KB regions (Q and dO, 64-column chunks 0 and 1)
-        // hold the eight 32 x 32 fp32 boxes: region b = d / 32, box row = query.
-        const uint32_t region = ((j / 32) < 2 ? sQ(st) : sdO(st)) + ((j / 32) & 1) * kChunkBytes + x * 8192;
-        const uint32_t stage_col = region + (j % 32) * 4;
+        const float2* nd = reinterpret_cast<const float2*>(smem + L::kStat + st * L::kStatBytes) + kTile / 2 + 32 * x;
 #pragma unroll
-        for (int q = 0; q < 64; ++q)
-          st_shared_f32(stage_col + (q / 32) * 4096 + (q % 32) * 128, __uint_as_float(dq[q]));
-        fence_proxy_async_smem();
-        named_bar_sync(3 + x, 128);
-        if (j == 0) {
-          for (int b = 0; b < 4; ++b) {
-            const uint32_t reg = (b < 2 ? sQ(st) : sdO(st)) + (b & 1) * kChunkBytes + x * 8192;
-            for (int r = 0; r < 2; ++r)
-              tma_reduce_add_3d(&tmdQacc, reg + r * 4096, 32 * b, u.h, row_base + q0 + 64 * x + 32 * r);
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(tR2 + lane_off + 64 * x + 32 * c, dp);
+          tmem_wait_ld();
+          uint32_t dsp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 d2 =
+                __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[16 * c + i]);
+            const float2 ds = __fmul2_rn(make_float2(pf[32 * c + 2 * i], pf[32 * c + 2 * i + 1]), d2);
+            dsp[i] = pack_bf16(ds.x, ds.y);
           }
-          tma_store_commit();
-          tma_store_wait_read();
-          mbar_arrive(bar(RED_DONE + st));
+          tmem_st16(tR2 + lane_off + 64 * x + 16 * c, dsp);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(DS_READY));
+        if (qn >= 0) {
+          ok = p_step(n + 1, qn);
+          if (!ok) break;
         }
         ++n;
+        qt = qn;
       }
-      if (j == 0) tma_store_wait_all();  // every reduction has landed before the CTA retires
     }
-    // the last reductions read Q stage rows the epilogue below overwrites
-    named_bar_sync(1, 256);
     // ---------------------------------------------------------- epilogue: dK, dV
     bool have = kvalid && ok && n > 0;
     if (have) {
       have = s2_wait(bar(ACC_DONE), 0, abort_flag, status, 32);
       tc_fence_after();
     }
-    const bool key_valid = have && (k0 + j < p.n_valid);
+    const bool key_valid = k0 + j < p.n_valid;
     const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t tsrc = which == 0 ? tdV : tdK;
-      const float mul = which == 0 ? 1.f : scale;
-      const uint32_t stage = sQ(which);
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const int d0 = x * 64 + 32 * c2;
-        uint32_t v[32];
-        if (have) {
-          tmem_ld32(tsrc + lane_off + d0, v);
-          tmem_wait_ld();
-        }
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = d0 + 8 * q;
-          const int chunk = col / 64, piece = (col % 64) / 8;
-          uint32_t w[4];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float a = key_valid ? __uint_as_float(v[8 * q + 2 * t]) * mul : 0.f;
-            const float b = key_valid ? __uint_as_float(v[8 * q + 2 * t + 1]) * mul : 0.f;
-            w[t] = pack_bf16(a, b);
-          }
-          st_shared_v4(stage + chunk * kChunkBytes + j * 128 + ((piece ^ (j & 7)) << 4), w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
+    // staging: dV -> Q stage 0, dK -> Q stage 1 (every MMA reading them has completed)
+    acc_to_smem<D>(tdV, lane_off, x, j, have, key_valid, 1.f, sQ(0));
+    acc_to_smem<D>(tdK, lane_off, x, j, have, key_valid, scale, sQ(1));
     fence_proxy_async_smem();
     named_bar_sync(2, 256);
     if (threadIdx.x == 0) {
@@ -797,45 +452,343 @@ __global__ void __launch_bounds__(bwds::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+#undef bar
+#undef sQ
+#undef sdO
 }
+
+// ------------------------------------------------------------------ dQ pass
+// Tensor memory (512 columns): S0, S1 [0, 256) double-buffered scores (then
+// dS as bf16 pairs in the first half of each warpgroup's 64 columns);
+// dP [256, 384); dQ [384, 384 + D).  Key tiles j of the unit, in order; the
+// issue order (one thread of warp 9) is
+//   S(0), S(1), dP(0), then per j:  dQ += dS(j) K(j),  dP(j+1),  S(j+2)
+// so the exponentials of tile j+1 overlap dQ(j) and dP(j+1).  K tiles live in
+// a ring of three slots (K(j) is read by S(j) and, two tiles later, dQ(j)),
+// V tiles in a ring of two.  Elementwise thread = query row (TMEM lane),
+// warpgroup x = key columns [64x, 64x + 64).
+namespace dqp {
+
+constexpr int kKSlots = 3, kVSlots = 2;
+enum Bar {
+  Q_FULL = 0,
+  K_FULL = 1,    // + slot (3)
+  K_EMPTY = 4,   // + slot (3)
+  V_FULL = 7,    // + slot (2)
+  V_EMPTY = 9,   // + slot (2)
+  S_FULL = 11,   // + buffer (2)
+  DP_FULL = 13,
+  DS_READY = 14,
+  DQ_DONE = 15,
+  NUM_BARS = 16
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kTileBytes = kTile * D * 2;
+  static constexpr int kQ = 0;
+  static constexpr int kdO = kTileBytes;
+  static constexpr int kK = 2 * kTileBytes;                // + slot * kTileBytes
+  static constexpr int kV = kK + kKSlots * kTileBytes;      // + slot * kTileBytes
+  static constexpr int kBars = kV + kVSlots * kTileBytes;
+  static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
+};
+
+}  // namespace dqp
+
+template <int D>
+__global__ void __launch_bounds__(bwd::kThreads, 1)
+    s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                     const __grid_constant__ CUtensorMap tmdQ, const Plan p, const float* __restrict__ delta,
+                     const float* __restrict__ lse2, int* __restrict__ status) {
+  using namespace bwd;
+  using namespace dqp;
+  using L = dqp::Layout<D>;
+  constexpr int kChunks = D / 64;
+
+  Unit u;
+  if (!decode_q_unit(p, blockIdx.x, u)) return;
+  extern __shared__ __align__(1024) uint8_t smem_dq[];
+  if (smem_u32(smem_dq) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(status, 256);
+    return;
+  }
+  const int qt = u.t[0];
+  const int q0 = tile_orig(p, u, qt);
+  const bool qvalid = u.part[0];  // the query tile holds a valid row
+
+  uint8_t* smem = smem_dq;
+  const uint32_t sb = smem_u32(smem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t sbar = sb + L::kBars;
+#define bar(i) (sbar + 8u * (uint32_t)(i))
+#define sKs(slot) (sb + L::kK + (uint32_t)(slot) * L::kTileBytes)
+#define sVs(slot) (sb + L::kV + (uint32_t)(slot) * L::kTileBytes)
+  const uint32_t sQ = sb + L::kQ, sdO = sb + L::kdO;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    mbar_init(bar(Q_FULL), 1);
+    for (int i = 0; i < kKSlots; ++i) {
+      mbar_init(bar(K_FULL + i), 1);
+      mbar_init(bar(K_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kVSlots; ++i) {
+      mbar_init(bar(V_FULL + i), 1);
+      mbar_init(bar(V_EMPTY + i), 1);
+    }
+    mbar_init(bar(S_FULL + 0), 1);
+    mbar_init(bar(S_FULL + 1), 1);
+    mbar_init(bar(DP_FULL), 1);
+    mbar_init(bar(DS_READY), 256);
+    mbar_init(bar(DQ_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tDP = tmem + 256, tdQ = tmem + 384;
+  const int row_base = u.b * p.N;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && qvalid) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(bar(Q_FULL), 2 * L::kTileBytes);
+      for (int c = 0; c < kChunks; ++c) {
+        tma_load_3d(sQ + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(Q_FULL));
+        tma_load_3d(sdO + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(Q_FULL));
+      }
+      int eK = 0, eV = 0;
+      bool ok = true;
+      auto load = [&](bool isK, int k) {
+        if (!ok) return;
+        const int e = isK ? eK : eV, slots = isK ? kKSlots : kVSlots;
+        const int slot = e % slots;
+        const uint32_t full = bar((isK ? K_FULL : V_FULL) + slot), empty = bar((isK ? K_EMPTY : V_EMPTY) + slot);
+        if (e >= slots) ok = s2_wait(empty, ((e / slots) - 1) & 1, abort_flag, status, 1);
+        if (!ok) return;
+        mbar_arrive_expect_tx(full, L::kTileBytes);
+        const uint32_t dst = isK ? sKs(slot) : sVs(slot);
+        const int row = row_base + tile_orig(p, u, k);
+        for (int c = 0; c < kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, isK ? &tmK : &tmV, c * 64, u.h, row, full);
+        if (isK) ++eK; else ++eV;
+      };
+      // consumption order: K(0), K(1), V(0), then per j: V(j+1), K(j+2)
+      int ka = next_k(p, u, -1);
+      int kb = ka >= 0 ? next_k(p, u, ka) : -1;
+      int kc = kb >= 0 ? next_k(p, u, kb) : -1;
+      if (ka >= 0) load(true, ka);
+      if (kb >= 0) load(true, kb);
+      if (ka >= 0) load(false, ka);
+      while (ok && ka >= 0) {
+        if (kb >= 0) load(false, kb);
+        if (kc >= 0) load(true, kc);
+        ka = kb;
+        kb = kc;
+        kc = kc >= 0 ? next_k(p, u, kc) : -1;
+      }
+      // the last loads must land before the CTA retires
+      for (int d = (eK > kKSlots ? eK - kKSlots : 0); d < eK; ++d)
+        s2_wait(bar(K_FULL + d % kKSlots), (d / kKSlots) & 1, abort_flag, status, 1);
+      for (int d = (eV > kVSlots ? eV - kVSlots : 0); d < eV; ++d)
+        s2_wait(bar(V_FULL + d % kVSlots), (d / kVSlots) & 1, abort_flag, status, 1);
+      s2_wait(bar(Q_FULL), 0, abort_flag, status, 1);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && qvalid) {
+      constexpr uint32_t id_s = umma_idesc_bf16(128, 128, 0, 0);  // S, dP: M queries, N keys, K-major
+      constexpr uint32_t id_q = umma_idesc_bf16(128, D, 0, 1);    // dQ: A = dS from TMEM, B = K MN-major
+      const uint64_t dQ_km = umma_desc_sw128(sQ, 16, 1024), ddO_km = umma_desc_sw128(sdO, 16, 1024);
+      const uint64_t dK_km = umma_desc_sw128(sKs(0), 16, 1024), dV_km = umma_desc_sw128(sVs(0), 16, 1024);
+      const uint64_t dK_mn = umma_desc_sw128(sKs(0), kChunkBytes, 1024);
+      constexpr uint64_t kSlotStep = (uint64_t)(L::kTileBytes >> 4);
+      int T = 0;  // key tiles of this unit
+      for (int k = next_k(p, u, -1); k >= 0; k = next_k(p, u, k)) ++T;
+      bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
+      auto issue_s = [&](int jj) {  // S(jj) = Q K(jj)^T -> S buffer jj % 2
+        const int slot = jj % kKSlots;
+        ok = ok && s2_wait(bar(K_FULL + slot), (jj / kKSlots) & 1, abort_flag, status, 2);
+        if (!ok) return;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)slot * kSlotStep;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + 128 * (jj % 2), dQ_km + S2_KM_OFF(kk), dK_km + so + S2_KM_OFF(kk), id_s, kk > 0);
+        umma_commit(bar(S_FULL + (jj % 2)));
+      };
+      auto issue_dp = [&](int jj) {  // dP(jj) = dO V(jj)^T -> dP
+        const int slot = jj % kVSlots;
+        ok = ok && s2_wait(bar(V_FULL + slot), (jj / kVSlots) & 1, abort_flag, status, 2);
+        if (!ok) return;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)slot * kSlotStep;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tDP, ddO_km + S2_KM_OFF(kk), dV_km + so + S2_KM_OFF(kk), id_s, kk > 0);
+        umma_commit(bar(DP_FULL));
+        umma_commit(bar(V_EMPTY + slot));
+      };
+      if (T > 0) issue_s(0);
+      if (T > 1) issue_s(1);
+      if (T > 0) issue_dp(0);
+      for (int jj = 0; ok && jj < T; ++jj) {
+        ok = s2_wait(bar(DS_READY), jj & 1, abort_flag, status, 2);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ += dS(jj) K(jj): K = 128 keys, 16 per step, dS pairs at S + 64·(kk/4) + 8·(kk%4)
+        const int slot = jj % kKSlots;
+        const uint64_t so = (uint64_t)slot * kSlotStep;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ts(tdQ, tmem + 128 * (jj % 2) + 64 * (kk / 4) + 8 * (kk % 4), dK_mn + so + S2_MN_OFF(kk), id_q,
+                  (jj > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(K_EMPTY + slot));
+        if (jj + 1 < T) issue_dp(jj + 1);  // dP(jj) was read before DS_READY(jj)
+        if (jj + 2 < T) issue_s(jj + 2);   // behind dQ(jj), the last reader of this S buffer
+      }
+      // every issued MMA must be complete before TMEM is read or released
+      umma_commit(bar(DQ_DONE));
+      s2_wait(bar(DQ_DONE), 0, abort_flag, status, 2);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ elementwise warpgroups
+    const int x = warp / 4;                // key columns [64x, 64x + 64)
+    const int r = (warp % 4) * 32 + lane;  // query row == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    const bool row_valid = q0 + r < p.n_valid;
+    bool ok = true;
+    int jj = 0;
+    if (qvalid) {
+      const size_t stat_at = ((size_t)u.b * p.H + u.h) * p.N + q0 + r;
+      const float nl = lse2[stat_at], nd = delta[stat_at];  // -lse·log2(e) (-inf if padded), -Delta
+      const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+      const float2 nl2 = make_float2(nl, nl), nd2 = make_float2(nd, nd);
+      for (int k = next_k(p, u, -1); ok && k >= 0; k = next_k(p, u, k), ++jj) {
+        const uint32_t tS = tmem + 128 * (jj % 2);
+        // key columns [0, lim) of this tile are visible from row r (causal diagonal, padding)
+        const int lim = col_limit(p, u, qt, k, r);
+        const bool masked = !__all_sync(0xffffffffu, lim == kTile);
+        ok = s2_wait(bar(S_FULL + (jj % 2)), (jj / 2) & 1, abort_flag, status, 4);
+        if (!ok) break;
+        tc_fence_after();
+        float pf[64];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(tS + lane_off + 64 * x + 32 * c, sv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 a = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl2);
+            float p0 = ex2(a.x), p1 = ex2(a.y);
+            if (masked) {
+              const int col = 64 * x + 32 * c + 2 * i;
+              p0 = col < lim ? p0 : 0.f;
+              p1 = col + 1 < lim ? p1 : 0.f;
+            }
+            pf[32 * c + 2 * i] = p0;
+            pf[32 * c + 2 * i + 1] = p1;
+          }
+        }
+        ok = s2_wait(bar(DP_FULL), jj & 1, abort_flag, status, 4);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(tDP + lane_off + 64 * x + 32 * c, dp);
+          tmem_wait_ld();
+          uint32_t dsp[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd2);
+            const float2 ds = __fmul2_rn(make_float2(pf[32 * c + 2 * i], pf[32 * c + 2 * i + 1]), d2);
+            dsp[i] = pack_bf16(ds.x, ds.y);
+          }
+          // dS pairs of key columns [32c, 32c + 32) -> S columns 64x + [16c, 16c + 16), already read
+          tmem_st16(tS + lane_off + 64 * x + 16 * c, dsp);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(DS_READY));
+      }
+    }
+    // ---------------------------------------------------------- epilogue: dq
+    bool have = qvalid && ok && jj > 0;
+    if (have) {
+      have = s2_wait(bar(DQ_DONE), 0, abort_flag, status, 4);
+      tc_fence_after();
+    }
+    const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
+    // staging in the Q tile (every MMA reading it has completed)
+    acc_to_smem<D>(tdQ, lane_off, x, r, have, row_valid, scale, sQ);
+    fence_proxy_async_smem();
+    named_bar_sync(2, 256);
+    if (threadIdx.x == 0) {
+      for (int c = 0; c < kChunks; ++c) tma_store_3d(&tmdQ, sQ + c * kChunkBytes, c * 64, u.h, row_base + q0);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+#undef bar
+#undef sKs
+#undef sVs
+}
+
+#undef S2_KM_OFF
+#undef S2_MN_OFF
 
 template <int D>
 int launch_bwd_impl(const BwdArgs& a, int stages) {
-  using L = bwd::Layout<D>;
-  static_assert(L::kAlloc <= 232448, "shared memory budget");
+  static_assert(dkdv::Layout<D>::kBytes <= 232448 && dqp::Layout<D>::kBytes <= 232448, "shared memory budget");
   const Plan& p = a.plan;
   const long long rows = (long long)p.B * p.N * p.H;
   cudaError_t e;
-  if (stages & 1) {  // prepare: Delta, lse2, zeroed dq accumulator
+  if (stages & 1) {  // prepare: -Delta and -lse·log2(e)
     constexpr int kRowsPerBlock = 256 / (D / 8);
     s2_bwd_pre<D><<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, a.stream>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.delta, a.lse2,
         p.B, p.N, p.H, p.n_valid);
-    e = cudaMemsetAsync(a.dq_acc, 0, (size_t)rows * D * sizeof(float), a.stream);
-    if (e != cudaSuccess) return (int)e;
-  }
-  if (stages & 2) {  // main: dK, dV and the dq accumulator
-    const int grid = grid_bwd(p);
-    if (D == 128) {
-      static_assert(bwds::Layout::kBytes <= 232448, "shared memory budget");
-      e = cudaFuncSetAttribute(s2_bwd_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwds::Layout::kBytes);
-      if (e != cudaSuccess) return (int)e;
-      s2_bwd_split_kernel<<<grid, bwds::kThreads, bwds::Layout::kBytes, a.stream>>>(
-          *a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK, *a.tmdV, *a.tmdQacc, p, a.delta, a.lse2, a.status);
-    } else {
-      e = cudaFuncSetAttribute(s2_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
-      if (e != cudaSuccess) return (int)e;
-      s2_bwd_kernel<D><<<grid, bwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK,
-                                                                     *a.tmdV, p, a.delta, a.lse2, a.dq_acc, a.status);
-    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;
   }
-  if (stages & 4) {  // finish: dq = bf16(scale * accumulator)
-    const long long n4 = rows * D / 4;
-    const float scale = p.scale_log2 * 0.69314718055994531f;
-    s2_bwd_dq_convert<<<148 * 8, 256, 0, a.stream>>>(reinterpret_cast<const float4*>(a.dq_acc),
-                                                    static_cast<uint2*>(a.dq), n4, scale);
+  const int grid = grid_bwd(p);
+  if (stages & 2) {  // dK, dV
+    constexpr int kBytes = dkdv::Layout<D>::kBytes;
+    e = cudaFuncSetAttribute(s2_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    if (e != cudaSuccess) return (int)e;
+    s2_bwd_dkdv_kernel<D><<<grid, bwd::kThreads, kBytes, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK,
+                                                                    *a.tmdV, p, a.delta, a.lse2, a.status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return (int)e;
+  }
+  if (stages & 4) {  // dQ
+    constexpr int kBytes = dqp::Layout<D>::kBytes;
+    e = cudaFuncSetAttribute(s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    if (e != cudaSuccess) return (int)e;
+    s2_bwd_dq_kernel<D><<<grid, bwd::kThreads, kBytes, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdQ, p,
+                                                                  a.delta, a.lse2, a.status);
   }
   return (int)cudaGetLastError();
 }

@@ -42,7 +42,7 @@ struct Plan {
   int nunit[2];    // max work units (pairs of q tiles) per segment, per class
   int ranks;       // max over classes of nseg * nunit (forward grid = ranks * B * H)
   int ntile[2];    // max tiles per segment, per class
-  int kv_ranks;    // max over classes of nseg * ntile (backward grid = kv_ranks * B * H)
+  int kv_ranks;    // max over classes of nseg * ntile (grid of each backward pass = kv_ranks * B * H)
   int hg_fwd, hg_bwd;  // heads interleaved per group of consecutive CTAs (L2 locality)
   float scale_log2;  // log2(e) / sqrt(D)
 };
@@ -198,6 +198,32 @@ S2_HD bool decode_kv_unit(const Plan& p, int L, Unit& u) {
   u.part[0] = tile_orig(p, u, kt) < p.n_valid;
   u.part[1] = false;
   u.kmax = u.ntiles - 1;
+  return true;
+}
+
+// Decode a linear dq-pass work index: one query tile of a segment, whose key
+// tiles run from the segment start to the diagonal (query tiles with the
+// most key tiles first).  Unit: t[0] = query tile, part[0] = it holds a valid
+// row, kmax = t[0].
+S2_HD bool decode_q_unit(const Plan& p, int L, Unit& u) {
+  int bh, r;
+  if (!split_index(p, L, p.kv_ranks, p.hg_bwd, bh, r)) return false;
+  u.b = bh / p.H;
+  u.h = bh % p.H;
+  u.cls = head_class(p, u.h);
+  const int S = p.nseg[u.cls], NT = p.ntile[u.cls];
+  if (r >= S * NT) return false;
+  const int rank = r / S, seg = r % S;
+  int len;
+  seg_bounds(p, u.cls, seg, u.vbeg, len);
+  u.ntiles = len / kTile;
+  const int qt = u.ntiles - 1 - rank;
+  if (qt < 0) return false;
+  u.t[0] = qt;
+  u.t[1] = -1;
+  u.part[0] = tile_orig(p, u, qt) < p.n_valid;
+  u.part[1] = false;
+  u.kmax = qt;
   return true;
 }
 

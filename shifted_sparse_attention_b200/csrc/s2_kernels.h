@@ -26,21 +26,19 @@ struct BwdArgs {
   const CUtensorMap* tmdO;
   const CUtensorMap* tmdK;
   const CUtensorMap* tmdV;
-  const CUtensorMap* tmdQacc;  // fp32 dq accumulator, box 32 x 1 x 32, no swizzle
+  const CUtensorMap* tmdQ;
   Plan plan;
   const void* o;      // bf16 [B, N, H, D]
   const void* dout;   // bf16 [B, N, H, D]
   const float* lse;   // [B, H, N]
   float* delta;       // workspace [B, H, N]: -(dout_i·o_i)
   float* lse2;        // workspace [B, H, N]: -lse_i·log2(e), -inf on padded rows
-  float* dq_acc;      // workspace [B, N, H, D] fp32
-  void* dq;           // bf16 [B, N, H, D]
   int* status;
   cudaStream_t stream;
 };
 
 int launch_fwd(const FwdArgs& a);
-// stages: 1 = prepare (Delta, lse2, zero accumulator), 2 = main, 4 = dq convert.
+// stages: 1 = prepare (Delta, lse2), 2 = dK/dV pass, 4 = dQ pass.
 int launch_bwd(const BwdArgs& a, int stages);
 // Sets the calling thread's s2attn_last_error() message; returns `code`.
 int report_error(int code, const char* fmt, ...);

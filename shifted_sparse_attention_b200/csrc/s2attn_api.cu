@@ -128,19 +128,6 @@ int make_tmap(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int6
   return S2_OK;
 }
 
-// The fp32 dq accumulator [B*N, H, D] for bulk reductions: box = 32 columns x 1 head x 32 rows.
-int make_tmap_acc(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t H, int64_t D) {
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(B * N)};
-  cuuint64_t strides[2] = {(cuuint64_t)(D * 4), (cuuint64_t)(H * D * 4)};
-  cuuint32_t box[3] = {32, 1, 32};
-  cuuint32_t elem[3] = {1, 1, 1};
-  CUresult r = st->encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, elem,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(S2_ERR_CUDA, "cuTensorMapEncodeTiled (accumulator) failed (%d)", (int)r);
-  return S2_OK;
-}
-
 int launch_status(int rc, const char* what) {
   if (rc == 0) return S2_OK;
   return fail(S2_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString((cudaError_t)rc));
@@ -163,7 +150,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 100; }
+int s2attn_version(void) { return 101; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -194,15 +181,15 @@ int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
   return s2attn_fwd_v(q, k, v, o, lse, B, N, H, D, G, N, variant, stream);
 }
 
-// Workspace = [Delta: B*H*N f32][lse*log2(e): B*H*N f32][dq accumulator: B*N*H*D f32],
-// each part starting on a 256-byte boundary.
+// Workspace = [-Delta: B*H*N f32][-lse*log2(e): B*H*N f32], each part starting
+// on a 256-byte boundary.
 static size_t stat_bytes(int64_t B, int64_t N, int64_t H) {
   return ((size_t)B * H * N * sizeof(float) + 255) / 256 * 256;
 }
 
 size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
   if (B < 1 || N < 1 || H < 1 || D < 1) return 0;
-  return 2 * stat_bytes(B, N, H) + (size_t)B * N * H * D * sizeof(float);
+  return 2 * stat_bytes(B, N, H);
 }
 
 int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -224,13 +211,14 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
     return fail(S2_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
-  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
   if ((rc = make_tmap(st, &tq, q, B, N, H, D)) || (rc = make_tmap(st, &tk, k, B, N, H, D)) ||
       (rc = make_tmap(st, &tv, v, B, N, H, D)) || (rc = make_tmap(st, &tdo, dout, B, N, H, D)) ||
-      (rc = make_tmap(st, &tdk, dk, B, N, H, D)) || (rc = make_tmap(st, &tdv, dv, B, N, H, D)))
+      (rc = make_tmap(st, &tdk, dk, B, N, H, D)) || (rc = make_tmap(st, &tdv, dv, B, N, H, D)) ||
+      (rc = make_tmap(st, &tdq, dq, B, N, H, D)))
     return rc;
   s2::BwdArgs a;
-  a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmdO = &tdo; a.tmdK = &tdk; a.tmdV = &tdv;
+  a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmdO = &tdo; a.tmdK = &tdk; a.tmdV = &tdv; a.tmdQ = &tdq;
   a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
   a.o = o;
   a.dout = dout;
@@ -238,11 +226,6 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
   const size_t sb = stat_bytes(B, N, H);
   a.delta = static_cast<float*>(workspace);
   a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
-  a.dq_acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * sb);
-  CUtensorMap tacc;
-  if ((rc = make_tmap_acc(st, &tacc, a.dq_acc, B, N, H, D))) return rc;
-  a.tmdQacc = &tacc;
-  a.dq = dq;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");

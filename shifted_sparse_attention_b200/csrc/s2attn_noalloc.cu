@@ -18,9 +18,8 @@
 // made before any stream capture starts.  Every call shares the one array, so
 // calls whose kernels overlap on the GPU (different streams, or different
 // host threads on one device) race on it.  The array keeps whatever the last
-// call left in it; the backward's prepare stage rewrites all of it that is
-// read (row statistics) or accumulated (the dq accumulator is cleared to
-// zero with cudaMemsetAsync, which allocates nothing).
+// call left in it; the backward's prepare stage rewrites every row statistic
+// the later stages read, so nothing has to be cleared.
 #include <cuda_runtime.h>
 
 #include <mutex>
