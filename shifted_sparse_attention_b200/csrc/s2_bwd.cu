@@ -146,31 +146,39 @@ __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restric
 // so the exponentials of tile n+1 overlap dK(n) and dP(n+1), and dS(n)
 // overlaps dV(n) and S(n+1).  Elementwise thread = key row j (TMEM lane),
 // warpgroup x = query columns [64x, 64x + 64); order P(0), [dS(n), P(n+1)].
+// Q tiles (with their -lse2 rows) live in a ring of three slots, dO tiles
+// (with their -Delta rows) in a ring of two: a slot is refilled as soon as
+// its last reader is done (dK for Q; dV and the dS step for dO), which puts
+// about six tile products between a load and its first use -- the L2's
+// latency under full load is of that order.
 namespace dkdv {
 
-constexpr int kStages = 2;
+constexpr int kQSlots = 3, kOSlots = 2;
 enum Bar {
   KV_FULL = 0,
-  QD_FULL = 1,   // + stage (2)
-  QD_EMPTY = 3,  // + stage (2)
-  S_FULL = 5,
-  DP_FULL = 6,
-  P_READY = 7,
-  DS_READY = 8,
-  ACC_DONE = 9,
-  NUM_BARS = 10
+  Q_FULL = 1,    // + slot (3)
+  Q_EMPTY = 4,   // + slot (3)
+  O_FULL = 7,    // + slot (2)
+  O_EMPTY = 9,   // + slot (2): dV's commit + the 256 elementwise threads after their dS step
+  S_FULL = 11,
+  DP_FULL = 12,
+  P_READY = 13,
+  DS_READY = 14,
+  ACC_DONE = 15,
+  NUM_BARS = 16
 };
 
 template <int D>
 struct Layout {
   static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kStatBytes = 2 * kTile * 4;  // -lse2[128], -Delta[128] of a query tile
+  static constexpr int kRowBytes = kTile * 4;  // one float32 statistic of a query tile
   static constexpr int kK = 0;
   static constexpr int kV = kTileBytes;
-  static constexpr int kQ = 2 * kTileBytes;               // + stage * kTileBytes
-  static constexpr int kdO = kQ + kStages * kTileBytes;   // + stage * kTileBytes
-  static constexpr int kStat = kdO + kStages * kTileBytes;  // + stage * kStatBytes
-  static constexpr int kBars = kStat + kStages * kStatBytes;
+  static constexpr int kQ = 2 * kTileBytes;                  // + slot * kTileBytes
+  static constexpr int kdO = kQ + kQSlots * kTileBytes;      // + slot * kTileBytes
+  static constexpr int kLse = kdO + kOSlots * kTileBytes;    // -lse2 rows, + slot * kRowBytes
+  static constexpr int kDelta = kLse + kQSlots * kRowBytes;  // -Delta rows, + slot * kRowBytes
+  static constexpr int kBars = kDelta + kOSlots * kRowBytes;
   static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
 };
 
@@ -213,9 +221,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
     mbar_init(bar(KV_FULL), 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(bar(QD_FULL + i), 1);
-      mbar_init(bar(QD_EMPTY + i), 1);
+    for (int i = 0; i < kQSlots; ++i) {
+      mbar_init(bar(Q_FULL + i), 1);
+      mbar_init(bar(Q_EMPTY + i), 1);
+    }
+    for (int i = 0; i < kOSlots; ++i) {
+      mbar_init(bar(O_FULL + i), 1);
+      mbar_init(bar(O_EMPTY + i), 1 + 256);
     }
     mbar_init(bar(S_FULL), 1);
     mbar_init(bar(DP_FULL), 1);
@@ -251,23 +263,27 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       int n = 0;
       bool ok = true;
       for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt)) {
-        const int st = n % kStages;
-        if (n >= kStages) ok = s2_wait(bar(QD_EMPTY + st), ((n / kStages) - 1) & 1, abort_flag, status, 8);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(QD_FULL + st), 2 * L::kTileBytes + L::kStatBytes);
         const int q0 = tile_orig(p, u, qt);
-        for (int c = 0; c < kChunks; ++c) {
-          tma_load_3d(sQ(st) + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
-          tma_load_3d(sdO(st) + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(QD_FULL + st));
-        }
-        const uint32_t sstat = sb + L::kStat + st * L::kStatBytes;
-        bulk_load(sstat, lse2 + stat_base + q0, kTile * 4, bar(QD_FULL + st));
-        bulk_load(sstat + kTile * 4, delta + stat_base + q0, kTile * 4, bar(QD_FULL + st));
+        const int sq = n % kQSlots, so = n % kOSlots;
+        if (n >= kQSlots) ok = s2_wait(bar(Q_EMPTY + sq), ((n / kQSlots) - 1) & 1, abort_flag, status, 8);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(Q_FULL + sq), L::kTileBytes + L::kRowBytes);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(sQ(sq) + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(Q_FULL + sq));
+        bulk_load(sb + L::kLse + sq * L::kRowBytes, lse2 + stat_base + q0, L::kRowBytes, bar(Q_FULL + sq));
+        if (n >= kOSlots) ok = s2_wait(bar(O_EMPTY + so), ((n / kOSlots) - 1) & 1, abort_flag, status, 8);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(O_FULL + so), L::kTileBytes + L::kRowBytes);
+        for (int c = 0; c < kChunks; ++c)
+          tma_load_3d(sdO(so) + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(O_FULL + so));
+        bulk_load(sb + L::kDelta + so * L::kRowBytes, delta + stat_base + q0, L::kRowBytes, bar(O_FULL + so));
         ++n;
       }
       // the last loads must land before the CTA retires
-      for (int d = (n > kStages ? n - kStages : 0); d < n; ++d)
-        s2_wait(bar(QD_FULL + d % kStages), (d / kStages) & 1, abort_flag, status, 8);
+      for (int d = (n > kQSlots ? n - kQSlots : 0); d < n; ++d)
+        s2_wait(bar(Q_FULL + d % kQSlots), (d / kQSlots) & 1, abort_flag, status, 8);
+      for (int d = (n > kOSlots ? n - kOSlots : 0); d < n; ++d)
+        s2_wait(bar(O_FULL + d % kOSlots), (d / kOSlots) & 1, abort_flag, status, 8);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -280,9 +296,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const uint64_t dQ_km = umma_desc_sw128(sQ(0), 16, 1024), ddO_km = umma_desc_sw128(sdO(0), 16, 1024);
       const uint64_t dQ_mn = umma_desc_sw128(sQ(0), kChunkBytes, 1024);
       const uint64_t ddO_mn = umma_desc_sw128(sdO(0), kChunkBytes, 1024);
-      constexpr uint64_t kStageStep = (uint64_t)(L::kTileBytes >> 4);
+      constexpr uint64_t kSlotStep = (uint64_t)(L::kTileBytes >> 4);
       bool ok = s2_wait(bar(KV_FULL), 0, abort_flag, status, 16);
-      if (ok) ok = s2_wait(bar(QD_FULL + 0), 0, abort_flag, status, 16);
+      if (ok) ok = s2_wait(bar(Q_FULL + 0), 0, abort_flag, status, 16);
       tc_fence_after();
       if (ok) {  // S(0)
 #pragma unroll
@@ -290,14 +306,15 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         umma_commit(bar(S_FULL));
       }
       int n = 0;
+      if (ok) ok = s2_wait(bar(O_FULL + 0), 0, abort_flag, status, 16);
+      int qn = next_q(p, u, kt);
       for (int qt = kt; ok && qt >= 0;) {
-        const int st = n % kStages;
-        const uint64_t so = (uint64_t)st * kStageStep;
-        const int qn = next_q(p, u, qt);
-        // dP^T(n) -> R2
+        const int sq = n % kQSlots, sd = n % kOSlots;
+        const uint64_t oq = (uint64_t)sq * kSlotStep, od = (uint64_t)sd * kSlotStep;
+        // dP^T(n) -> R2 (dO(n) has landed)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tR2, dV_km + S2_KM_OFF(kk), ddO_km + so + S2_KM_OFF(kk), id_s, kk > 0);
+          umma_ss(tR2, dV_km + S2_KM_OFF(kk), ddO_km + od + S2_KM_OFF(kk), id_s, kk > 0);
         umma_commit(bar(DP_FULL));
         // dV += P^T(n) dO(n): K = 128 queries, 16 per step, P^T pairs at R1 + 64·(kk/4) + 8·(kk%4)
         ok = s2_wait(bar(P_READY), n & 1, abort_flag, status, 16);
@@ -305,19 +322,26 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tdV, tR1 + 64 * (kk / 4) + 8 * (kk % 4), ddO_mn + so + S2_MN_OFF(kk), id_acc,
+          umma_ts(tdV, tR1 + 64 * (kk / 4) + 8 * (kk % 4), ddO_mn + od + S2_MN_OFF(kk), id_acc,
                   (n > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(O_EMPTY + sd));  // dV is the last MMA reading dO(n)
         // S^T(n+1) -> R1
         if (qn >= 0) {
-          const int st1 = (n + 1) % kStages;
-          ok = s2_wait(bar(QD_FULL + st1), ((n + 1) / kStages) & 1, abort_flag, status, 16);
+          const int sq1 = (n + 1) % kQSlots;
+          ok = s2_wait(bar(Q_FULL + sq1), ((n + 1) / kQSlots) & 1, abort_flag, status, 16);
           if (!ok) break;
-          tc_fence_after();
-          const uint64_t so1 = (uint64_t)st1 * kStageStep;
+          const uint64_t oq1 = (uint64_t)sq1 * kSlotStep;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(tR1, dK_km + S2_KM_OFF(kk), dQ_km + so1 + S2_KM_OFF(kk), id_s, kk > 0);
+            umma_ss(tR1, dK_km + S2_KM_OFF(kk), dQ_km + oq1 + S2_KM_OFF(kk), id_s, kk > 0);
           umma_commit(bar(S_FULL));
+        }
+        // the next tile and its dO, while S(n+1) is queued
+        const int qnn = qn >= 0 ? next_q(p, u, qn) : -1;
+        if (qn >= 0) {
+          const int sd1 = (n + 1) % kOSlots;
+          ok = s2_wait(bar(O_FULL + sd1), ((n + 1) / kOSlots) & 1, abort_flag, status, 16);
+          if (!ok) break;
         }
         // dK += dS^T(n) Q(n), dS^T pairs at R2 + 64·(kk/4) + 8·(kk%4)
         ok = s2_wait(bar(DS_READY), n & 1, abort_flag, status, 16);
@@ -325,11 +349,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ts(tdK, tR2 + 64 * (kk / 4) + 8 * (kk % 4), dQ_mn + so + S2_MN_OFF(kk), id_acc,
+          umma_ts(tdK, tR2 + 64 * (kk / 4) + 8 * (kk % 4), dQ_mn + oq + S2_MN_OFF(kk), id_acc,
                   (n > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(QD_EMPTY + st));
+        umma_commit(bar(Q_EMPTY + sq));
         ++n;
         qt = qn;
+        qn = qnn;
       }
       // every issued MMA must be complete before TMEM is read or released
       umma_commit(bar(ACC_DONE));
@@ -349,16 +374,16 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       float pf[64];  // P of the current tile (fp32), from its exponentials to its dS
       // P(nn): S^T -> P^T (bf16 pairs into R1) and pf
       auto p_step = [&](int nn, int qtile) -> bool {
-        const int st = nn % kStages;
+        const int sq = nn % kQSlots;
         // masks on the diagonal tile and on a key tile with padding; padded
         // queries are zeroed by their -inf statistic
         const bool masked = (qtile == kt) || key_tile_ragged;
         int lo = 0, hi = kTile;
         if (masked) query_range(p, u, kt, qtile, j, lo, hi);
-        if (!s2_wait(bar(QD_FULL + st), (nn / kStages) & 1, abort_flag, status, 32)) return false;
+        if (!s2_wait(bar(Q_FULL + sq), (nn / kQSlots) & 1, abort_flag, status, 32)) return false;
         if (!s2_wait(bar(S_FULL), nn & 1, abort_flag, status, 32)) return false;
         tc_fence_after();
-        const float2* nl = reinterpret_cast<const float2*>(smem + L::kStat + st * L::kStatBytes) + 32 * x;
+        const float2* nl = reinterpret_cast<const float2*>(smem + L::kLse + sq * L::kRowBytes) + 32 * x;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {  // 32 query columns at a time
           uint32_t sv[32];
@@ -390,13 +415,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       int qt = kt;
       ok = p_step(0, qt);
       while (ok && qt >= 0) {
-        const int st = n % kStages;
+        const int sd = n % kOSlots;
         const int qn = next_q(p, u, qt);
         // dS(n) = P (dP - Delta) -> dS^T pairs into R2
-        ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
+        ok = s2_wait(bar(O_FULL + sd), (n / kOSlots) & 1, abort_flag, status, 32);
+        if (ok) ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
         if (!ok) break;
         tc_fence_after();
-        const float2* nd = reinterpret_cast<const float2*>(smem + L::kStat + st * L::kStatBytes) + kTile / 2 + 32 * x;
+        const float2* nd = reinterpret_cast<const float2*>(smem + L::kDelta + sd * L::kRowBytes) + 32 * x;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
@@ -415,6 +441,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(DS_READY));
+        mbar_arrive(bar(O_EMPTY + sd));  // done with the -Delta rows of dO slot sd
         if (qn >= 0) {
           ok = p_step(n + 1, qn);
           if (!ok) break;
@@ -431,7 +458,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     }
     const bool key_valid = k0 + j < p.n_valid;
     const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
-    // staging: dV -> Q stage 0, dK -> Q stage 1 (every MMA reading them has completed)
+    // staging: dV -> Q slot 0, dK -> Q slot 1 (every MMA reading them has completed)
     acc_to_smem<D>(tdV, lane_off, x, j, have, key_valid, 1.f, sQ(0));
     acc_to_smem<D>(tdK, lane_off, x, j, have, key_valid, scale, sQ(1));
     fence_proxy_async_smem();
@@ -618,22 +645,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       int T = 0;  // key tiles of this unit
       for (int k = next_k(p, u, -1); k >= 0; k = next_k(p, u, k)) ++T;
       bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
-      auto issue_s = [&](int jj) {  // S(jj) = Q K(jj)^T -> S buffer jj % 2
+      auto issue_s = [&](int jj) {  // S(jj) = Q K(jj)^T -> S buffer jj % 2 (K(jj) has landed)
         const int slot = jj % kKSlots;
-        ok = ok && s2_wait(bar(K_FULL + slot), (jj / kKSlots) & 1, abort_flag, status, 2);
         if (!ok) return;
-        tc_fence_after();
         const uint64_t so = (uint64_t)slot * kSlotStep;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
           umma_ss(tmem + 128 * (jj % 2), dQ_km + S2_KM_OFF(kk), dK_km + so + S2_KM_OFF(kk), id_s, kk > 0);
         umma_commit(bar(S_FULL + (jj % 2)));
       };
-      auto issue_dp = [&](int jj) {  // dP(jj) = dO V(jj)^T -> dP
+      auto issue_dp = [&](int jj) {  // dP(jj) = dO V(jj)^T -> dP (V(jj) has landed)
         const int slot = jj % kVSlots;
-        ok = ok && s2_wait(bar(V_FULL + slot), (jj / kVSlots) & 1, abort_flag, status, 2);
         if (!ok) return;
-        tc_fence_after();
         const uint64_t so = (uint64_t)slot * kSlotStep;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
@@ -641,11 +664,21 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         umma_commit(bar(DP_FULL));
         umma_commit(bar(V_EMPTY + slot));
       };
-      if (T > 0) issue_s(0);
-      if (T > 1) issue_s(1);
-      if (T > 0) issue_dp(0);
+      auto wait_k = [&](int jj) {
+        ok = ok && s2_wait(bar(K_FULL + jj % kKSlots), (jj / kKSlots) & 1, abort_flag, status, 2);
+      };
+      auto wait_v = [&](int jj) {
+        ok = ok && s2_wait(bar(V_FULL + jj % kVSlots), (jj / kVSlots) & 1, abort_flag, status, 2);
+      };
+      if (T > 0) { wait_k(0); issue_s(0); }
+      if (T > 1) { wait_k(1); issue_s(1); }
+      if (T > 0) { wait_v(0); issue_dp(0); }
       for (int jj = 0; ok && jj < T; ++jj) {
-        ok = s2_wait(bar(DS_READY), jj & 1, abort_flag, status, 2);
+        // the loads this iteration consumes first (landed long ago, as a rule), then the
+        // dS hand-off: the three batches below then issue back to back
+        if (jj + 1 < T) wait_v(jj + 1);
+        if (jj + 2 < T) wait_k(jj + 2);
+        if (ok) ok = s2_wait(bar(DS_READY), jj & 1, abort_flag, status, 2);
         if (!ok) break;
         tc_fence_after();
         // dQ += dS(jj) K(jj): K = 128 keys, 16 per step, dS pairs at S + 64·(kk/4) + 8·(kk%4)

@@ -15,11 +15,16 @@
 //   warp  8    TMA producer: Q tiles once, then the K/V stream
 //   warp  9    TMEM allocator and tcgen05.mma issuer (one thread)
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A and O_B at 256 + x·D.
-// Shared memory: Q_A, Q_B, a ring of three K/V slots, P_A, P_B; all tiles
-// are 128-byte-swizzled, 1024-byte aligned, as TMA writes and UMMA reads them.
-// MMA order per key tile k (software pipelined so that the tensor core works
-// on the next S while the softmax warps exponentiate the current one):
-//     S_A(k+1)=Q_A K(k+1)^T, S_B(k+1)=Q_B K(k+1)^T, O_A += P_A(k) V(k), O_B += P_B(k) V(k)
+// The softmax writes P (bf16 pairs) over the first 64 columns of its S, and
+// O += P V reads it from there as the A operand: P never touches shared
+// memory, whose bandwidth the score MMAs (both operands in shared memory)
+// already use in full.  Shared memory: Q_A, Q_B and a ring of five K/V slots;
+// all tiles are 128-byte-swizzled, 1024-byte aligned, as TMA writes and UMMA
+// reads them.  MMA order per key tile k:
+//     O_A += P_A(k) V(k), S_A(k+1) = Q_A K(k+1)^T, O_B += P_B(k) V(k), S_B(k+1)
+// so each softmax warpgroup works on its tile while the tensor core runs the
+// other tile's two products, and S_x(k+1) overwrites P_x(k) only behind the
+// MMA that reads it.
 // Softmax uses base-2 exponentials with a lazily updated running max: O and
 // l are rescaled only when the row max grows by more than 8 (a factor 256),
 // which keeps bf16 P and fp32 sums exact enough and skips most rescales.
@@ -36,16 +41,14 @@ namespace s2 {
 namespace fwd {
 
 constexpr int kThreads = 320;
-constexpr int kSlots = 3;
+constexpr int kSlots = 5;
 constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16 = one 128B-swizzle column block
 
 enum Bar {
-  KV_FULL = 0,      // + slot (3)
-  KV_EMPTY = 3,     // + slot (3)
-  S_FULL = 6,       // + tile (2)
-  S_FREE = 8,       // + tile (2)
-  P_FULL = 10,      // + tile (2)
-  PV_DONE = 12,     // + tile (2)
+  KV_FULL = 0,      // + slot (5)
+  KV_EMPTY = 5,     // + slot (5)
+  S_FULL = 10,      // + tile (2)
+  P_FULL = 12,      // + tile (2)
   Q_FULL = 14,
   MMA_DONE = 15,
   NUM_BARS = 16
@@ -55,11 +58,9 @@ template <int D>
 struct Layout {
   static constexpr int kQBytes = kTile * D * 2;
   static constexpr int kKVBytes = kTile * D * 2;
-  static constexpr int kPBytes = kTile * kTile * 2;
   static constexpr int kQ = 0;
   static constexpr int kKV = 2 * kQBytes;
-  static constexpr int kP = kKV + kSlots * kKVBytes;
-  static constexpr int kBars = kP + 2 * kPBytes;
+  static constexpr int kBars = kKV + kSlots * kKVBytes;
   static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
@@ -84,6 +85,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 
   Unit u;
   if (!decode_unit(p, blockIdx.x, u)) return;
+  // The two query tiles as scalars: indexing u.t[] / u.part[] with a runtime
+  // tile number would put the whole struct in local memory.
+  const int tA = u.t[0], tB = u.t[1];
+  const bool pA = u.part[0], pB = u.part[1];
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -97,7 +102,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #define bar(i) (sbar + 8u * (uint32_t)(i))
 #define sQ(x) (sb + L::kQ + (uint32_t)(x) * L::kQBytes)
 #define sKV(slot) (sb + L::kKV + (uint32_t)(slot) * L::kKVBytes)
-#define sP(x) (sb + L::kP + (uint32_t)(x) * L::kPBytes)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   if (threadIdx.x == 0) {
@@ -107,9 +111,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(S_FULL + x), 1);
-      mbar_init(bar(S_FREE + x), 128);
       mbar_init(bar(P_FULL + x), 128);
-      mbar_init(bar(PV_DONE + x), 1);
     }
     mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(MMA_DONE), 1);
@@ -134,11 +136,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       uint32_t qbytes = 0;
-      for (int x = 0; x < 2; ++x) qbytes += u.part[x] ? L::kQBytes : 0;
+      qbytes += pA ? L::kQBytes : 0;
+      qbytes += pB ? L::kQBytes : 0;
       mbar_arrive_expect_tx(bar(Q_FULL), qbytes);
+#pragma unroll
       for (int x = 0; x < 2; ++x) {
-        if (!u.part[x]) continue;
-        const int row = row_base + tile_orig(p, u, u.t[x]);
+        if (!(x ? pB : pA)) continue;
+        const int row = row_base + tile_orig(p, u, x ? tB : tA);
         for (int c = 0; c < kChunks; ++c)
           tma_load_3d(sQ(x) + c * kChunkBytes, &tmQ, c * 64, u.h, row, bar(Q_FULL));
       }
@@ -154,13 +158,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           tma_load_3d(sKV(slot) + c * kChunkBytes, tm, c * 64, u.h, row, bar(KV_FULL + slot));
         ++e;
       };
+      // consumption order: K(k0), then per key tile V(k), K(next k)
       int kc = next_k(p, u, -1);
       if (kc >= 0) load(&tmK, kc);
       while (ok && kc >= 0) {
         const int kn = next_k(p, u, kc);
-        if (kn >= 0) load(&tmK, kn);
-        if (!ok) break;
         load(&tmV, kc);
+        if (!ok) break;
+        if (kn >= 0) load(&tmK, kn);
         kc = kn;
       }
       // drain: the last loads must land before the CTA retires
@@ -185,67 +190,74 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   } while (0)
 #define ISSUE_PV(x, slot, acc)                                                                    \
   do {                                                                                            \
-    const uint64_t a0_ = umma_desc_sw128(sP(x), 16, 1024);                                        \
     const uint64_t b0_ = umma_desc_sw128(sKV(slot), kChunkBytes, 1024);                           \
     _Pragma("unroll") for (int kk = 0; kk < kTile / 16; ++kk) {                                   \
-      const uint64_t aoff_ = ((kk / 4) * kChunkBytes + (kk % 4) * 32) >> 4;                        \
-      umma_ss(tmem + 256 + (x) * D, a0_ + aoff_, b0_ + (uint64_t)(kk * 2048 >> 4), idesc_pv,      \
-              ((acc) || kk > 0) ? 1u : 0u);                                                       \
+      umma_ts(tmem + 256 + (x) * D, tmem + (x) * 128 + 8 * kk, b0_ + (uint64_t)(kk * 2048 >> 4),   \
+              idesc_pv, ((acc) || kk > 0) ? 1u : 0u);                                             \
     }                                                                                             \
   } while (0)
       bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
-      int nqk[2] = {0, 0}, npv[2] = {0, 0};
-      int e = 0;
+      int npvA = 0, npvB = 0;
+      int e = 0;  // position in the K/V load sequence
       int kc = next_k(p, u, -1);
       if (ok && kc >= 0) {
         const int eK = e++;
         ok = s2_wait(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
-        tc_fence_after();
-        for (int x = 0; ok && x < 2; ++x)
-          if (tile_takes(p, u, x, kc)) {
-            ISSUE_QK(x, eK % kSlots);
-            umma_commit(bar(S_FULL + x));
-            ++nqk[x];
-          }
+        if (ok && pA && kc <= tA) {
+          ISSUE_QK(0, eK % kSlots);
+          umma_commit(bar(S_FULL + 0));
+        }
+        if (ok && pB && kc <= tB) {
+          ISSUE_QK(1, eK % kSlots);
+          umma_commit(bar(S_FULL + 1));
+        }
         umma_commit(bar(KV_EMPTY + eK % kSlots));
       }
+      // loads of the first iteration: V(kc) and K(next)
+      int kn = kc >= 0 ? next_k(p, u, kc) : -1;
+      int eV = e++;
+      int eK = kn >= 0 ? e++ : -1;
+      if (ok && kc >= 0) ok = s2_wait(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
+      if (ok && kn >= 0) ok = s2_wait(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
       while (ok && kc >= 0) {
-        const int kn = next_k(p, u, kc);
-        const int eK = (kn >= 0) ? e++ : -1;
-        const int eV = e++;
-        if (kn >= 0) {
-          ok = s2_wait(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
+        // per tile: O_x += P_x(kc) V(kc), then S_x(kn) into the same TMEM columns
+        const int sV = eV % kSlots, sK = eK % kSlots;
+        if (pA && kc <= tA) {
+          ok = s2_wait(bar(P_FULL + 0), npvA & 1, abort_flag, status, 2);
           if (!ok) break;
           tc_fence_after();
-        }
-        // Both next-tile score MMAs first, then both PV MMAs: a late P on one
-        // query tile never holds back the other tile's next S.
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (kn >= 0 && tile_takes(p, u, x, kn)) {
-            if (nqk[x] > 0) ok = s2_wait(bar(S_FREE + x), (nqk[x] - 1) & 1, abort_flag, status, 2);
-            if (!ok) break;
-            tc_fence_after();
-            ISSUE_QK(x, eK % kSlots);
-            umma_commit(bar(S_FULL + x));
-            ++nqk[x];
+          ISSUE_PV(0, sV, npvA > 0);
+          ++npvA;
+          if (kn >= 0 && kn <= tA) {
+            ISSUE_QK(0, sK);
+            umma_commit(bar(S_FULL + 0));
           }
         }
+        // The next iteration's tile and loads, while tile A's products are queued:
+        // the issuing thread's bookkeeping then never leaves the tensor core idle.
+        const int knn = kn >= 0 ? next_k(p, u, kn) : -1;
+        const int eV2 = kn >= 0 ? e++ : -1;   // V(kn)
+        const int eK2 = knn >= 0 ? e++ : -1;  // K(knn)
+        if (eV2 >= 0) ok = s2_wait(bar(KV_FULL + eV2 % kSlots), (eV2 / kSlots) & 1, abort_flag, status, 2);
+        if (ok && eK2 >= 0) ok = s2_wait(bar(KV_FULL + eK2 % kSlots), (eK2 / kSlots) & 1, abort_flag, status, 2);
         if (!ok) break;
-        if (kn >= 0) umma_commit(bar(KV_EMPTY + eK % kSlots));
-        ok = s2_wait(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (tile_takes(p, u, x, kc)) {
-            ok = s2_wait(bar(P_FULL + x), npv[x] & 1, abort_flag, status, 2);
-            if (!ok) break;
-            tc_fence_after();
-            ISSUE_PV(x, eV % kSlots, npv[x] > 0);
-            umma_commit(bar(PV_DONE + x));
-            ++npv[x];
+        if (pB && kc <= tB) {
+          ok = s2_wait(bar(P_FULL + 1), npvB & 1, abort_flag, status, 2);
+          if (!ok) break;
+          tc_fence_after();
+          ISSUE_PV(1, sV, npvB > 0);
+          ++npvB;
+          if (kn >= 0 && kn <= tB) {
+            ISSUE_QK(1, sK);
+            umma_commit(bar(S_FULL + 1));
           }
         }
-        if (!ok) break;
-        umma_commit(bar(KV_EMPTY + eV % kSlots));
+        umma_commit(bar(KV_EMPTY + sV));
+        if (kn >= 0) umma_commit(bar(KV_EMPTY + sK));
         kc = kn;
+        kn = knn;
+        eV = eV2;
+        eK = eK2;
       }
       // every issued MMA must be complete before TMEM is released
       umma_commit(bar(MMA_DONE));
@@ -260,14 +272,16 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + x * 128;
     const uint32_t tO = tmem + lane_off + 256 + x * D;
-    if (u.t[x] >= 0) {
-      const int q0 = tile_orig(p, u, u.t[x]);
+    const int tx = x ? tB : tA;
+    const bool px = x ? pB : pA;
+    if (tx >= 0) {
+      const int q0 = tile_orig(p, u, tx);
       const bool row_valid = (q0 + r) < p.n_valid;
       float m_used = -INFINITY, l = 0.f;
       int n = 0;
       bool ok = true;
-      if (u.part[x]) {
-        for (int k = 0; k <= u.t[x] && ok; ++k) {
+      if (px) {
+        for (int k = 0; k <= tx && ok; ++k) {
           if (!ktile_valid(p, u, k)) continue;
           ok = s2_wait(bar(S_FULL + x), n & 1, abort_flag, status, 4);
           if (!ok) break;
@@ -276,12 +290,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[j * 32]));
           tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(bar(S_FREE + x));
 
           // Masks (the causal triangle of the diagonal tile, padded keys or rows)
           // only where some row of the warp needs them.
-          const int lim = col_limit(p, u, u.t[x], k, r);
+          const int lim = col_limit(p, u, tx, k, r);
           if (!__all_sync(0xffffffffu, lim == kTile)) {
 #pragma unroll
             for (int c = 0; c < kTile; ++c)
@@ -323,10 +335,8 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           const float2 acct = __fadd2_rn(acc01, acc23);
           l += acct.x + acct.y;
 
+          // S_x(k) was issued behind O_x += P_x(k-1) V(k-1), so O_x is complete here
           if (n > 0) {
-            ok = s2_wait(bar(PV_DONE + x), (n - 1) & 1, abort_flag, status, 4);
-            if (!ok) break;
-            tc_fence_after();
             if (__any_sync(0xffffffffu, need)) {
               const float f = need ? factor : 1.f;
 #pragma unroll
@@ -341,24 +351,21 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
               tmem_wait_st();
             }
           }
-          // P (bf16) -> shared memory, K-major, 128B swizzle
-#pragma unroll
-          for (int pc = 0; pc < 16; ++pc) {
-            const uint32_t addr = sP(x) + (pc / 8) * kChunkBytes + r * 128 + (((pc % 8) ^ (r & 7)) << 4);
-            st_shared_v4(addr, s[pc * 4], s[pc * 4 + 1], s[pc * 4 + 2], s[pc * 4 + 3]);
-          }
-          fence_proxy_async_smem();
+          // P (bf16 pairs) -> TMEM columns [0, 64) of S_x, the A operand of O_x += P_x V
+          tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
+          tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
+          tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(P_FULL + x));
           ++n;
         }
-        if (ok && n > 0) {
-          ok = s2_wait(bar(PV_DONE + x), (n - 1) & 1, abort_flag, status, 4);
+        if (ok && n > 0) {  // the last O_x += P_x V has completed
+          ok = s2_wait(bar(MMA_DONE), 0, abort_flag, status, 4);
           tc_fence_after();
         }
       }
       // ---------------------------------------------------------- epilogue
-      const bool have = u.part[x] && ok && n > 0;
+      const bool have = px && ok && n > 0;
       const float inv_l = (have && row_valid) ? 1.f / l : 0.f;
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
@@ -374,7 +381,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         for (int pc = 0; pc < 4; ++pc) {
           const int col = j * 32 + pc * 8;  // first of 8 columns
           const int chunk = col / 64, piece = (col % 64) / 8;
-          const uint32_t addr = sP(x) + chunk * kChunkBytes + r * 128 + ((piece ^ (r & 7)) << 4);
+          const uint32_t addr = sQ(x) + chunk * kChunkBytes + r * 128 + ((piece ^ (r & 7)) << 4);
           const uint32_t* oo = &o[pc * 8];
           st_shared_v4(addr, pack_bf16(__uint_as_float(oo[0]) * inv_l, __uint_as_float(oo[1]) * inv_l),
                        pack_bf16(__uint_as_float(oo[2]) * inv_l, __uint_as_float(oo[3]) * inv_l),
@@ -388,7 +395,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       named_bar_sync(1 + x, 128);
       if (r == 0) {
         for (int c = 0; c < kChunks; ++c)
-          tma_store_3d(&tmO, sP(x) + c * kChunkBytes, c * 64, u.h, row_base + q0);
+          tma_store_3d(&tmO, sQ(x) + c * kChunkBytes, c * 64, u.h, row_base + q0);
         tma_store_commit();
         tma_store_wait_all();
       }
@@ -408,7 +415,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #undef bar
 #undef sQ
 #undef sKV
-#undef sP
 
 template <int D>
 int launch_fwd_impl(const FwdArgs& a) {

@@ -111,6 +111,10 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
+// After a wait that orders this thread behind other threads' tcgen05 loads or
+// stores (TMEM hand-offs).  Waits on TMA completion need no fence: the
+// tensor-memory copy engine and the MMA both act in the async proxy, ordered
+// by the mbarrier's transaction count.
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
