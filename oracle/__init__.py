@@ -70,10 +70,13 @@ def lib() -> ctypes.CDLL:
         L.s2o_adjacency_row.restype = None
         L.s2o_pair_count.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
         L.s2o_pair_count.restype = i64
-        L.s2o_attention.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, i64,
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        L.s2o_pair_count_docs.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int, i32p]
+        L.s2o_pair_count_docs.restype = i64
+        L.s2o_attention.argtypes = [u16p, u16p, u16p, u16p, i32p, i64, i64, i64, i64, i64, i64,
                                     ctypes.c_int, i64, i64, i64p, i64, dp, dp, dp, dp, dp]
         L.s2o_attention.restype = ctypes.c_int
-        L.s2o_attention_window.argtypes = [u16p, u16p, u16p, u16p, i64, i64, i64, i64, i64, i64,
+        L.s2o_attention_window.argtypes = [u16p, u16p, u16p, u16p, i32p, i64, i64, i64, i64, i64, i64,
                                            ctypes.c_int, i64, i64, i64p, i64, dp, dp, dp, dp, dp]
         L.s2o_attention_window.restype = ctypes.c_int
         L.s2o_num_threads.argtypes = []
@@ -108,6 +111,31 @@ def pair_count(N: int, G: int, n_valid: int, variant: int, head_class: int) -> i
     return int(lib().s2o_pair_count(N, G, n_valid, variant, head_class))
 
 
+def pair_count_docs(N: int, G: int, n_valid: int, variant: int, head_class: int, doc) -> int:
+    """Visible pairs of one head class under a document mask (doc: N per-position IDs)."""
+    d = np.ascontiguousarray(np.asarray(doc, dtype=np.int32))
+    assert d.shape == (N,)
+    return int(lib().s2o_pair_count_docs(N, G, n_valid, variant, head_class, _ptr(d, ctypes.c_int32)))
+
+
+def _docs(doc, B: int, N: int):
+    """Per-position document IDs as a contiguous int32 [B, N] array (None: one document)."""
+    if doc is None:
+        return None
+    try:
+        import torch
+
+        if isinstance(doc, torch.Tensor):
+            doc = doc.detach().cpu().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    d = np.ascontiguousarray(np.asarray(doc, dtype=np.int32))
+    if d.shape == (N,):
+        d = np.ascontiguousarray(np.broadcast_to(d, (B, N)))
+    assert d.shape == (B, N), d.shape
+    return d
+
+
 def num_threads() -> int:
     return int(lib().s2o_num_threads())
 
@@ -124,7 +152,7 @@ def _bits(x) -> np.ndarray:
 
 
 def attention(q, k, v, dout=None, *, G: int, variant: int, n_valid: int | None = None,
-              rows: tuple[int, int] | None = None, heads=None):
+              rows: tuple[int, int] | None = None, heads=None, doc=None):
     """Run the oracle.
 
     q, k, v, dout: bf16 [B, N, H, D] (torch tensors or uint16 bit arrays).
@@ -132,10 +160,12 @@ def attention(q, k, v, dout=None, *, G: int, variant: int, n_valid: int | None =
     is given, dq, dk, dv.  Only rows in ``rows`` (default all) and heads in
     ``heads`` (flattened b*H+h, default all) are computed; entries outside
     are NaN (o, lse, dq) or hold only the processed rows' contributions
-    (dk, dv).
+    (dk, dv).  ``doc``: per-position document IDs [B, N] or [N] (document
+    mask of packed sequences), or None.
     """
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, N, H, D = qb.shape
+    dd = _docs(doc, B, N)
     nv = N if n_valid is None else int(n_valid)
     r0, r1 = (0, N) if rows is None else rows
     o = np.full((B, N, H, D), np.nan)
@@ -153,6 +183,7 @@ def attention(q, k, v, dout=None, *, G: int, variant: int, n_valid: int | None =
     rc = lib().s2o_attention(
         _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
         _ptr(gb, ctypes.c_uint16) if want_bwd else None,
+        _ptr(dd, ctypes.c_int32) if dd is not None else None,
         B, N, H, D, G, nv, variant, r0, r1, hp, nh,
         _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
         _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double),
@@ -166,7 +197,7 @@ def attention(q, k, v, dout=None, *, G: int, variant: int, n_valid: int | None =
 
 
 def attention_window(q, k, v, dout=None, *, G: int, variant: int, rows: tuple[int, int], heads,
-                     n_valid: int | None = None):
+                     n_valid: int | None = None, doc=None):
     """The oracle on query rows [r0, r1) of the given heads (flattened b*H+h),
     with compact outputs: o, dq, dk, dv [len(heads), r1 - r0, D]; lse
     [len(heads), r1 - r0].  dk / dv hold the contributions of the window's rows
@@ -176,6 +207,7 @@ def attention_window(q, k, v, dout=None, *, G: int, variant: int, rows: tuple[in
     B, N, H, D = qb.shape
     nv = N if n_valid is None else int(n_valid)
     r0, r1 = rows
+    dd = _docs(doc, B, N)
     harr = np.ascontiguousarray(np.asarray(heads, dtype=np.int64))
     nh, W = len(harr), r1 - r0
     o = np.full((nh, W, D), np.nan)
@@ -188,6 +220,7 @@ def attention_window(q, k, v, dout=None, *, G: int, variant: int, rows: tuple[in
     rc = lib().s2o_attention_window(
         _ptr(qb, ctypes.c_uint16), _ptr(kb, ctypes.c_uint16), _ptr(vb, ctypes.c_uint16),
         _ptr(gb, ctypes.c_uint16) if want_bwd else None,
+        _ptr(dd, ctypes.c_int32) if dd is not None else None,
         B, N, H, D, G, nv, variant, r0, r1, _ptr(harr, ctypes.c_int64), nh,
         _ptr(o, ctypes.c_double), _ptr(lse, ctypes.c_double),
         _ptr(dq, ctypes.c_double), _ptr(dk, ctypes.c_double), _ptr(dv, ctypes.c_double),

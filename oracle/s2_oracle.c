@@ -33,6 +33,11 @@
  *     invalid query rows see nothing: o = 0, lse = -inf, and their output
  *     gradient is treated as 0 (loss mask).
  *   - lse is the natural log of sum_j exp(scale q_i·k_j); scale = 1/sqrt(D).
+ *   - document mask ([PT] §1.1 "因果mask与样本packing"): when several documents
+ *     are packed into one sequence, j is visible from i only if, in addition,
+ *     doc(i) == doc(j); the same constraint applies to the original and the
+ *     shifted grouping.  doc is a per-position ID array [B, N] (NULL: one
+ *     document); IDs need not be contiguous runs here.
  */
 #include <math.h>
 #include <stdint.h>
@@ -103,6 +108,17 @@ int64_t s2o_pair_count(int64_t N, int64_t G, int64_t n_valid, int variant, int h
   return c;
 }
 
+/* Number of visible (i, j) pairs under a document mask (doc: [N] IDs of one
+ * batch row), by enumeration. */
+int64_t s2o_pair_count_docs(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                            const int32_t* doc) {
+  int64_t c = 0;
+  for (int64_t i = 0; i < N; ++i)
+    for (int64_t j = 0; j < N; ++j)
+      c += s2o_visible(N, G, n_valid, variant, head_class, i, j) && doc[i] == doc[j];
+  return c;
+}
+
 /* bf16 bit pattern -> double (exact). */
 static double bf16_to_double(uint16_t b) {
   uint32_t u = ((uint32_t)b) << 16;
@@ -124,6 +140,7 @@ static size_t at(int64_t N, int64_t H, int64_t D, int64_t b, int64_t i, int64_t 
  *   rows          : query rows [row_begin, row_end) are processed.
  *   heads         : list of flattened (b*H + h) heads to process, or NULL for
  *                   all B*H heads.
+ *   doc           : per-position document IDs [B, N], or NULL (one document).
  *   o, dq         : [B, N, H, D] float64, written for the processed rows.
  *   lse           : [B, H, N] float64, written for the processed rows.
  *   dk, dv        : [B, N, H, D] float64, ACCUMULATED (+=) with the
@@ -141,7 +158,7 @@ static size_t at(int64_t N, int64_t H, int64_t D, int64_t b, int64_t i, int64_t 
  *   dq_i = scale sum_j dS_ij k_j,  dk_j += scale dS_ij q_i,  dv_j += a_ij g_i.
  */
 int s2o_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
-                  int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
+                  const int32_t* doc, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
                   int variant, int64_t row_begin, int64_t row_end,
                   const int64_t* heads, int64_t n_heads,
                   double* o, double* lse, double* dq, double* dk, double* dv) {
@@ -167,7 +184,8 @@ int s2o_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const
       /* S_i: the visible keys of row i */
       int64_t ns = 0;
       for (int64_t j = 0; j < N; ++j)
-        if (s2o_visible(N, G, n_valid, variant, head_class, i, j)) js[ns++] = j;
+        if (s2o_visible(N, G, n_valid, variant, head_class, i, j) && (!doc || doc[b * N + i] == doc[b * N + j]))
+          js[ns++] = j;
 
       for (int64_t d = 0; d < D; ++d) qi[d] = bf16_to_double(q[at(N, H, D, b, i, h, d)]);
 
@@ -235,10 +253,11 @@ int s2o_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, const
  *   dk_w, dv_w [n_heads][r1 - r0][D]   keys r0..r1-1, ACCUMULATED from the
  *              window's rows only (exact for keys whose visible-from rows
  *              all lie inside the window; the caller zeroes them)
- * heads: flattened (b*H + h) list.  dout may be NULL (forward only).
+ * heads: flattened (b*H + h) list.  dout may be NULL (forward only); doc as
+ * for s2o_attention.
  */
 int s2o_attention_window(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
-                         int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
+                         const int32_t* doc, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
                          int variant, int64_t r0, int64_t r1, const int64_t* heads, int64_t n_heads,
                          double* o_w, double* lse_w, double* dq_w, double* dk_w, double* dv_w) {
   if (B < 1 || N < 1 || H < 2 || D < 1 || G < 2 || (H % 2) || (G % 2) || (N % G)) return -1;
@@ -262,7 +281,8 @@ int s2o_attention_window(const uint16_t* q, const uint16_t* k, const uint16_t* v
       const size_t wi = (size_t)(t * W + (i - r0));
       int64_t ns = 0;
       for (int64_t j = 0; j < N; ++j)
-        if (s2o_visible(N, G, n_valid, variant, head_class, i, j)) js[ns++] = j;
+        if (s2o_visible(N, G, n_valid, variant, head_class, i, j) && (!doc || doc[b * N + i] == doc[b * N + j]))
+          js[ns++] = j;
       for (int64_t d = 0; d < D; ++d) qi[d] = bf16_to_double(q[at(N, H, D, b, i, h, d)]);
       if (ns == 0) {
         for (int64_t d = 0; d < D; ++d) {
