@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--variant", type=int, default=None, help="0 strict, 1 rolled, 2 dense causal")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--doc-len", type=int, default=0,
+                    help="pack documents of this many tokens (document mask); reports exact-pair TFLOP/s")
     return ap.parse_args()
 
 
@@ -55,6 +57,24 @@ def peaks():
         return {"bf16_burst": d["bf16_tflops"], "bf16_sustained": d["bf16_tflops_sustained"],
                 "hbm_gbs": d["hbm_gbs"], "source": "measured"}
     return {"bf16_burst": 1590.0, "bf16_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def doc_pair_counts(w, variant, doc_len):
+    """Visited pairs per head class under a document mask of back-to-back documents of
+    doc_len tokens (strict or dense variant, no padding): every segment cut by the
+    document boundaries is a causal triangle."""
+    N, G = w.N, w.G
+    tri = lambda L: L * (L + 1) // 2
+    docs = set(range(0, N + 1, doc_len)) | {N}
+
+    def pairs(group_cuts):
+        c = sorted(docs | set(group_cuts))
+        return sum(tri(b - a) for a, b in zip(c, c[1:]))
+
+    if variant == 2:
+        return pairs({0, N}), pairs({0, N})
+    s = G // 2
+    return pairs(set(range(0, N + 1, G))), pairs({0, N} | set(range(s, N, G)))
 
 
 def pair_counts(w, variant):
@@ -281,20 +301,29 @@ def run_ours(args, rank, world, local_rank):
     ws = torch.empty(s2.s2attn_bwd_workspace_size(B, N, H, D), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     nv = w.n_valid
+    docs = None
+    if args.doc_len:
+        if variant == 1 or w.valid != N:
+            raise SystemExit("--doc-len supports the strict and dense variants without padding")
+        ids = (torch.arange(N, device=dev, dtype=torch.int32) // args.doc_len).expand(B, N).contiguous()
+        docs = s2.doc_bounds(ids)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        s2.forward(q, k, v, G, variant, nv, out=o, lse=lse)
+        s2.forward(q, k, v, G, variant, nv, out=o, lse=lse, docs=docs)
         if ev is not None:
             ev[1].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE,
+                    docs=docs)
         if ev is not None:
             ev[2].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DKDV)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DKDV,
+                    docs=docs)
         if ev is not None:
             ev[3].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ)
+        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ,
+                    docs=docs)
         if ev is not None:
             ev[4].record(stream)
 
@@ -368,7 +397,7 @@ def run_ours(args, rank, world, local_rank):
 
     # CPU oracle leg (rank 0, N = 1 only)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.doc_len:
         dt, fl, threads, desc = oracle_sample({n: x[n] for n in x}, w, variant, 256)
         cpu = {"value": fl / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
@@ -377,13 +406,17 @@ def run_ours(args, rank, world, local_rank):
         return
     pk = peaks()
     ms_step = ms / args.steps
-    flops_step = w.formula_flops(passes="fwd+bwd")
-    value = job_tflops(world, flops_step, ms_step)
-    pc = pair_counts(w, variant)
+    pc = doc_pair_counts(w, variant, args.doc_len) if args.doc_len else pair_counts(w, variant)
     if pc is not None:
         pairs = w.B * (w.H // 2) * (pc[0] + pc[1])
     else:
         pairs = None
+    # the metric's formula counts the grouping's causal work; under a document mask
+    # the useful work is the exact visited pairs (14·D FLOPs each, forward + backward)
+    flops_step = pairs * 14 * D if args.doc_len else w.formula_flops(passes="fwd+bwd")
+    value = job_tflops(world, flops_step, ms_step)
+    if e2e is not None and args.doc_len:
+        e2e["value"] = world * flops_step / (e2e["ms_per_step"] * 1e-3) / 1e12
     # dominant kernel: the longest of the forward, the dK/dV pass and the dQ pass.
     # Algorithmic FLOPs per visited pair: forward 4·D (Q K^T, P V); dK/dV pass
     # 8·D (S, dP, dV, dK); dQ pass 2·D (dQ only: its S and dP are recomputed).
@@ -401,10 +434,12 @@ def run_ours(args, rank, world, local_rank):
             "traffic": _traffic(kname, src),
             "algorithmic_flops_per_launch": algo, "avg_launch_ms": per[dom]}
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC + (" (document mask: exact visited pairs)" if args.doc_len else ""),
+        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": dict(_config(w, variant), parallelism="replicas%d" % world if world > 1 else "single"),
+        "config": dict(_config(w, variant), parallelism="replicas%d" % world if world > 1 else "single",
+                       **({"doc_len": args.doc_len} if args.doc_len else {})),
         "pct_of_peak": {"bf16_burst": value / world / pk["bf16_burst"],
                         "bf16_sustained": value / world / pk["bf16_sustained"],
                         "nominal_2250": value / world / 2250.0},

@@ -118,6 +118,32 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
                         int variant, void* workspace, size_t workspace_bytes, int stages,
                         void* stream);
 
+/* Packed sequences ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,
+ * "因果mask与样本packing"): when several documents are packed into one
+ * sequence, key j is visible from query i only if, in addition, both lie in
+ * the same document; the same constraint applies to the original and the
+ * shifted grouping, so that the shift never puts two documents into one group.
+ *
+ * The document mask is passed as per-position bounds: doc_bounds is int32
+ * [B, N, 2], device memory, 8-byte aligned, entry (b, x) = {first position,
+ * one past the last position} of the document holding original position x
+ * of batch row b.  Documents must be contiguous runs of positions.
+ * s2attn_doc_bounds computes the bounds from per-position document IDs
+ * (int32 [B, N]; a document is a maximal run of equal IDs).  Tile pairs that
+ * share no document are skipped, so packing many short documents also saves
+ * work.  Results are those of s2attn_fwd_v / s2attn_bwd_stages_v with the
+ * visibility additionally restricted to same-document pairs. */
+int s2attn_doc_bounds(const int32_t* doc_ids, int32_t* doc_bounds, int64_t B, int64_t N, void* stream);
+
+int s2attn_fwd_docs(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int32_t* doc_bounds, int64_t B, int64_t N, int64_t H, int64_t D, int64_t G,
+                    int64_t n_valid, int variant, void* stream);
+
+int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, const int32_t* doc_bounds, void* dq, void* dk, void* dv, int64_t B,
+                    int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                    void* workspace, size_t workspace_bytes, int stages, void* stream);
+
 /* Size of the fixed scratch array behind s2attn_bwd_noalloc_v (32 MiB). */
 #define S2_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -158,7 +184,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 101. */
+/* ABI version of this header (major*100 + minor): 102. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

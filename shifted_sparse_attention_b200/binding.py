@@ -31,6 +31,10 @@ SIGNATURES = {
                              _int, _vp, _sz, _int, _vp], _int),
     "s2attn_bwd_noalloc_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                               _int, _vp], _int),
+    "s2attn_doc_bounds": ([_vp, _vp, _i64, _i64, _vp], _int),
+    "s2attn_fwd_docs": ([_vp, _vp, _vp, _vp, _fp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
+    "s2attn_bwd_docs": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
+                         _int, _vp, _sz, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
@@ -127,6 +131,22 @@ def s2attn_bwd_noalloc_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_val
                                       _ptr(dk), _ptr(dv), B, N, H, D, G, n_valid, variant, _stream(stream))
 
 
+def s2attn_doc_bounds(doc_ids, doc_bounds, B, N, stream=None) -> int:
+    return lib().s2attn_doc_bounds(_ptr(doc_ids), _ptr(doc_bounds), B, N, _stream(stream))
+
+
+def s2attn_fwd_docs(q, k, v, o, lse, doc_bounds, B, N, H, D, G, n_valid, variant, stream=None) -> int:
+    return lib().s2attn_fwd_docs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(doc_bounds), B, N, H, D, G,
+                                 n_valid, variant, _stream(stream))
+
+
+def s2attn_bwd_docs(q, k, v, o, dout, lse, doc_bounds, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,
+                    workspace_bytes, stages, stream=None) -> int:
+    return lib().s2attn_bwd_docs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(doc_bounds),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G, n_valid, variant, _ptr(workspace),
+                                 workspace_bytes, stages, _stream(stream))
+
+
 def s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, out, stream=None) -> int:
     return lib().s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, _ptr(out), _stream(stream))
 
@@ -148,19 +168,42 @@ def _shape(q):
     return tuple(int(x) for x in q.shape)
 
 
-def forward(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None, out=None, lse=None, stream=None):
-    """S²-Attn forward; returns (o [B,N,H,D] bf16, lse [B,H,N] fp32)."""
+def doc_bounds(doc_ids, stream=None):
+    """Per-position document bounds [B, N, 2] (int32) from document IDs [B, N] (int32, CUDA)."""
+    if doc_ids.dim() != 2 or doc_ids.dtype != torch.int32 or not doc_ids.is_cuda or not doc_ids.is_contiguous():
+        raise ValueError("expected a contiguous CUDA int32 tensor [B, N] of document IDs")
+    B, N = (int(x) for x in doc_ids.shape)
+    out = torch.empty((B, N, 2), dtype=torch.int32, device=doc_ids.device)
+    _check(s2attn_doc_bounds(doc_ids, out, B, N, stream))
+    return out
+
+
+def _bounds(docs, B, N):
+    if docs.shape != (B, N, 2) or docs.dtype != torch.int32 or not docs.is_cuda or not docs.is_contiguous():
+        raise ValueError("expected contiguous CUDA int32 document bounds [B, N, 2] (see doc_bounds)")
+    return docs
+
+
+def forward(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None, out=None, lse=None, stream=None,
+            docs=None):
+    """S²-Attn forward; returns (o [B,N,H,D] bf16, lse [B,H,N] fp32).
+
+    docs: optional per-position document bounds [B, N, 2] (from doc_bounds) for
+    packed sequences."""
     B, N, H, D = _shape(q)
     nv = N if n_valid is None else int(n_valid)
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    _check(s2attn_fwd_v(q, k, v, o, l, B, N, H, D, G, nv, variant, stream))
+    if docs is None:
+        _check(s2attn_fwd_v(q, k, v, o, l, B, N, H, D, G, nv, variant, stream))
+    else:
+        _check(s2attn_fwd_docs(q, k, v, o, l, _bounds(docs, B, N), B, N, H, D, G, nv, variant, stream))
     return o, l
 
 
 def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int | None = None,
-             grads=None, workspace=None, stream=None, stages: int = 7):
-    """S²-Attn backward; returns (dq, dk, dv) bf16 [B,N,H,D]."""
+             grads=None, workspace=None, stream=None, stages: int = 7, docs=None):
+    """S²-Attn backward; returns (dq, dk, dv) bf16 [B,N,H,D].  docs as for forward."""
     B, N, H, D = _shape(q)
     nv = N if n_valid is None else int(n_valid)
     if grads is None:
@@ -169,8 +212,13 @@ def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int 
     ws_bytes = s2attn_bwd_workspace_size(B, N, H, D)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    _check(s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, nv, variant, workspace,
-                               workspace.numel() * workspace.element_size(), stages, stream))
+    wb = workspace.numel() * workspace.element_size()
+    if docs is None:
+        _check(s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, nv, variant, workspace, wb,
+                                   stages, stream))
+    else:
+        _check(s2attn_bwd_docs(q, k, v, o, dout, lse, _bounds(docs, B, N), dq, dk, dv, B, N, H, D, G, nv, variant,
+                               workspace, wb, stages, stream))
     return dq, dk, dv
 
 

@@ -47,17 +47,19 @@ constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16: one 128-byte
 #define S2_KM_OFF(kk) ((uint64_t)((((kk) / 4) * kChunkBytes + ((kk) % 4) * 32) >> 4))
 #define S2_MN_OFF(kk) ((uint64_t)(((kk) * 2048) >> 4))
 
-// Next query tile after qt (up to the segment end) that holds a valid row, or -1.
-__device__ __forceinline__ int next_q(const Plan& p, const Unit& u, int qt) {
+// Next query tile after qt (up to the segment end) that holds a valid row and
+// meets the span [lo, hi) of the documents touching the key tile, or -1.
+__device__ __forceinline__ int next_q(const Plan& p, const Unit& u, int qt, int lo, int hi) {
   for (int j = qt + 1; j <= u.kmax; ++j)
-    if (ktile_valid(p, u, j)) return j;
+    if (ktile_valid(p, u, j) && tile_meets(tile_orig(p, u, j), lo, hi)) return j;
   return -1;
 }
 
-// Next valid key tile after k (up to the query tile u.t[0]), or -1.
-__device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k) {
+// Next valid key tile after k (up to the query tile u.t[0]) that meets the
+// span [lo, hi) of the documents touching the query tile, or -1.
+__device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k, int lo, int hi) {
   for (int j = k + 1; j <= u.t[0]; ++j)
-    if (ktile_valid(p, u, j)) return j;
+    if (ktile_valid(p, u, j) && tile_meets(tile_orig(p, u, j), lo, hi)) return j;
   return -1;
 }
 
@@ -207,6 +209,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int kt = u.t[0];
   const int k0 = tile_orig(p, u, kt);
   const bool kvalid = u.part[0];
+  int lK, hK;  // span of the documents touching the key tile
+  doc_span(p, u.b, k0, lK, hK);
 
   uint8_t* smem = smem_kv;
   const uint32_t sb = smem_u32(smem);
@@ -262,7 +266,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
       int n = 0;
       bool ok = true;
-      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt)) {
+      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt, lK, hK)) {
         const int q0 = tile_orig(p, u, qt);
         const int sq = n % kQSlots, so = n % kOSlots;
         if (n >= kQSlots) ok = s2_wait(bar(Q_EMPTY + sq), ((n / kQSlots) - 1) & 1, abort_flag, status, 8);
@@ -307,7 +311,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
       int n = 0;
       if (ok) ok = s2_wait(bar(O_FULL + 0), 0, abort_flag, status, 16);
-      int qn = next_q(p, u, kt);
+      int qn = next_q(p, u, kt, lK, hK);
       for (int qt = kt; ok && qt >= 0;) {
         const int sq = n % kQSlots, sd = n % kOSlots;
         const uint64_t oq = (uint64_t)sq * kSlotStep, od = (uint64_t)sd * kSlotStep;
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           umma_commit(bar(S_FULL));
         }
         // the next tile and its dO, while S(n+1) is queued
-        const int qnn = qn >= 0 ? next_q(p, u, qn) : -1;
+        const int qnn = qn >= 0 ? next_q(p, u, qn, lK, hK) : -1;
         if (qn >= 0) {
           const int sd1 = (n + 1) % kOSlots;
           ok = s2_wait(bar(O_FULL + sd1), ((n + 1) / kOSlots) & 1, abort_flag, status, 16);
@@ -375,11 +379,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       // P(nn): S^T -> P^T (bf16 pairs into R1) and pf
       auto p_step = [&](int nn, int qtile) -> bool {
         const int sq = nn % kQSlots;
-        // masks on the diagonal tile and on a key tile with padding; padded
-        // queries are zeroed by their -inf statistic
-        const bool masked = (qtile == kt) || key_tile_ragged;
+        // masks on the diagonal tile, on a key tile with padding and under a
+        // document mask; padded queries are zeroed by their -inf statistic
+        const bool masked = (qtile == kt) || key_tile_ragged || p.docs != nullptr;
         int lo = 0, hi = kTile;
-        if (masked) query_range(p, u, kt, qtile, j, lo, hi);
+        if (masked) key_cols(p, u, kt, qtile, j, lo, hi);
         if (!s2_wait(bar(Q_FULL + sq), (nn / kQSlots) & 1, abort_flag, status, 32)) return false;
         if (!s2_wait(bar(S_FULL), nn & 1, abort_flag, status, 32)) return false;
         tc_fence_after();
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       ok = p_step(0, qt);
       while (ok && qt >= 0) {
         const int sd = n % kOSlots;
-        const int qn = next_q(p, u, qt);
+        const int qn = next_q(p, u, qt, lK, hK);
         // dS(n) = P (dP - Delta) -> dS^T pairs into R2
         ok = s2_wait(bar(O_FULL + sd), (n / kOSlots) & 1, abort_flag, status, 32);
         if (ok) ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
@@ -544,6 +548,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int qt = u.t[0];
   const int q0 = tile_orig(p, u, qt);
   const bool qvalid = u.part[0];  // the query tile holds a valid row
+  int lQ = 0, hQ = p.N;           // span of the documents touching the query tile
+  if (qvalid) doc_span(p, u.b, q0, lQ, hQ);
 
   uint8_t* smem = smem_dq;
   const uint32_t sb = smem_u32(smem);
@@ -612,9 +618,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (isK) ++eK; else ++eV;
       };
       // consumption order: K(0), K(1), V(0), then per j: V(j+1), K(j+2)
-      int ka = next_k(p, u, -1);
-      int kb = ka >= 0 ? next_k(p, u, ka) : -1;
-      int kc = kb >= 0 ? next_k(p, u, kb) : -1;
+      int ka = next_k(p, u, -1, lQ, hQ);
+      int kb = ka >= 0 ? next_k(p, u, ka, lQ, hQ) : -1;
+      int kc = kb >= 0 ? next_k(p, u, kb, lQ, hQ) : -1;
       if (ka >= 0) load(true, ka);
       if (kb >= 0) load(true, kb);
       if (ka >= 0) load(false, ka);
@@ -623,7 +629,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (kc >= 0) load(true, kc);
         ka = kb;
         kb = kc;
-        kc = kc >= 0 ? next_k(p, u, kc) : -1;
+        kc = kc >= 0 ? next_k(p, u, kc, lQ, hQ) : -1;
       }
       // the last loads must land before the CTA retires
       for (int d = (eK > kKSlots ? eK - kKSlots : 0); d < eK; ++d)
@@ -643,7 +649,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const uint64_t dK_mn = umma_desc_sw128(sKs(0), kChunkBytes, 1024);
       constexpr uint64_t kSlotStep = (uint64_t)(L::kTileBytes >> 4);
       int T = 0;  // key tiles of this unit
-      for (int k = next_k(p, u, -1); k >= 0; k = next_k(p, u, k)) ++T;
+      for (int k = next_k(p, u, -1, lQ, hQ); k >= 0; k = next_k(p, u, k, lQ, hQ)) ++T;
       bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
       auto issue_s = [&](int jj) {  // S(jj) = Q K(jj)^T -> S buffer jj % 2 (K(jj) has landed)
         const int slot = jj % kKSlots;
@@ -710,11 +716,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const float nl = lse2[stat_at], nd = delta[stat_at];  // -lse·log2(e) (-inf if padded), -Delta
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nl2 = make_float2(nl, nl), nd2 = make_float2(nd, nd);
-      for (int k = next_k(p, u, -1); ok && k >= 0; k = next_k(p, u, k), ++jj) {
+      for (int k = next_k(p, u, -1, lQ, hQ); ok && k >= 0; k = next_k(p, u, k, lQ, hQ), ++jj) {
         const uint32_t tS = tmem + 128 * (jj % 2);
-        // key columns [0, lim) of this tile are visible from row r (causal diagonal, padding)
-        const int lim = col_limit(p, u, qt, k, r);
-        const bool masked = !__all_sync(0xffffffffu, lim == kTile);
+        // key columns [cmin, cmax) of this tile are visible from row r (causal diagonal,
+        // padding, the row's document)
+        int cmin, cmax;
+        row_cols(p, u, qt, k, r, cmin, cmax);
+        const bool masked = !__all_sync(0xffffffffu, cmin == 0 && cmax == kTile);
         ok = s2_wait(bar(S_FULL + (jj % 2)), (jj / 2) & 1, abort_flag, status, 4);
         if (!ok) break;
         tc_fence_after();
@@ -730,8 +738,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             float p0 = ex2(a.x), p1 = ex2(a.y);
             if (masked) {
               const int col = 64 * x + 32 * c + 2 * i;
-              p0 = col < lim ? p0 : 0.f;
-              p1 = col + 1 < lim ? p1 : 0.f;
+              p0 = (col >= cmin && col < cmax) ? p0 : 0.f;
+              p1 = (col + 1 >= cmin && col + 1 < cmax) ? p1 : 0.f;
             }
             pf[32 * c + 2 * i] = p0;
             pf[32 * c + 2 * i + 1] = p1;

@@ -65,10 +65,18 @@ struct Layout {
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-// Smallest valid key tile > k (and <= kmax), or -1.
-__device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k) {
+// Query tile x (its index tx, whether it holds a valid row px, and the span
+// [lo, hi) of the documents touching it) takes part at key tile k.
+__device__ __forceinline__ bool takes(const Plan& p, const Unit& u, bool px, int tx, int lo, int hi, int k) {
+  return px && k <= tx && tile_meets(tile_orig(p, u, k), lo, hi);
+}
+
+// Smallest key tile > k that holds a valid key and that one of the unit's two
+// query tiles takes part at, or -1.
+__device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k, bool pA, int tA, int lA, int hA, bool pB,
+                                      int tB, int lB, int hB) {
   for (int j = k + 1; j <= u.kmax; ++j)
-    if (ktile_valid(p, u, j)) return j;
+    if (ktile_valid(p, u, j) && (takes(p, u, pA, tA, lA, hA, j) || takes(p, u, pB, tB, lB, hB, j))) return j;
   return -1;
 }
 
@@ -89,6 +97,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   // tile number would put the whole struct in local memory.
   const int tA = u.t[0], tB = u.t[1];
   const bool pA = u.part[0], pB = u.part[1];
+  // spans of the documents touching each query tile (everything without documents)
+  int lA = 0, hA = p.N, lB = 0, hB = p.N;
+  if (pA) doc_span(p, u.b, tile_orig(p, u, tA), lA, hA);
+  if (pB) doc_span(p, u.b, tile_orig(p, u, tB), lB, hB);
+#define NEXT_K(k) next_k(p, u, (k), pA, tA, lA, hA, pB, tB, lB, hB)
+#define TAKES_A(k) takes(p, u, pA, tA, lA, hA, (k))
+#define TAKES_B(k) takes(p, u, pB, tB, lB, hB, (k))
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -159,10 +174,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         ++e;
       };
       // consumption order: K(k0), then per key tile V(k), K(next k)
-      int kc = next_k(p, u, -1);
+      int kc = NEXT_K(-1);
       if (kc >= 0) load(&tmK, kc);
       while (ok && kc >= 0) {
-        const int kn = next_k(p, u, kc);
+        const int kn = NEXT_K(kc);
         load(&tmV, kc);
         if (!ok) break;
         if (kn >= 0) load(&tmK, kn);
@@ -199,22 +214,22 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = s2_wait(bar(Q_FULL), 0, abort_flag, status, 2);
       int npvA = 0, npvB = 0;
       int e = 0;  // position in the K/V load sequence
-      int kc = next_k(p, u, -1);
+      int kc = NEXT_K(-1);
       if (ok && kc >= 0) {
         const int eK = e++;
         ok = s2_wait(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
-        if (ok && pA && kc <= tA) {
+        if (ok && TAKES_A(kc)) {
           ISSUE_QK(0, eK % kSlots);
           umma_commit(bar(S_FULL + 0));
         }
-        if (ok && pB && kc <= tB) {
+        if (ok && TAKES_B(kc)) {
           ISSUE_QK(1, eK % kSlots);
           umma_commit(bar(S_FULL + 1));
         }
         umma_commit(bar(KV_EMPTY + eK % kSlots));
       }
       // loads of the first iteration: V(kc) and K(next)
-      int kn = kc >= 0 ? next_k(p, u, kc) : -1;
+      int kn = kc >= 0 ? NEXT_K(kc) : -1;
       int eV = e++;
       int eK = kn >= 0 ? e++ : -1;
       if (ok && kc >= 0) ok = s2_wait(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
@@ -222,35 +237,37 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       while (ok && kc >= 0) {
         // per tile: O_x += P_x(kc) V(kc), then S_x(kn) into the same TMEM columns
         const int sV = eV % kSlots, sK = eK % kSlots;
-        if (pA && kc <= tA) {
+        // (a tile's key tiles need not start together with the other tile's under a
+        // document mask: S_x(kn) is issued whenever x takes kn, behind any O_x += P_x V)
+        if (TAKES_A(kc)) {
           ok = s2_wait(bar(P_FULL + 0), npvA & 1, abort_flag, status, 2);
           if (!ok) break;
           tc_fence_after();
           ISSUE_PV(0, sV, npvA > 0);
           ++npvA;
-          if (kn >= 0 && kn <= tA) {
-            ISSUE_QK(0, sK);
-            umma_commit(bar(S_FULL + 0));
-          }
+        }
+        if (kn >= 0 && TAKES_A(kn)) {
+          ISSUE_QK(0, sK);
+          umma_commit(bar(S_FULL + 0));
         }
         // The next iteration's tile and loads, while tile A's products are queued:
         // the issuing thread's bookkeeping then never leaves the tensor core idle.
-        const int knn = kn >= 0 ? next_k(p, u, kn) : -1;
+        const int knn = kn >= 0 ? NEXT_K(kn) : -1;
         const int eV2 = kn >= 0 ? e++ : -1;   // V(kn)
         const int eK2 = knn >= 0 ? e++ : -1;  // K(knn)
         if (eV2 >= 0) ok = s2_wait(bar(KV_FULL + eV2 % kSlots), (eV2 / kSlots) & 1, abort_flag, status, 2);
         if (ok && eK2 >= 0) ok = s2_wait(bar(KV_FULL + eK2 % kSlots), (eK2 / kSlots) & 1, abort_flag, status, 2);
         if (!ok) break;
-        if (pB && kc <= tB) {
+        if (TAKES_B(kc)) {
           ok = s2_wait(bar(P_FULL + 1), npvB & 1, abort_flag, status, 2);
           if (!ok) break;
           tc_fence_after();
           ISSUE_PV(1, sV, npvB > 0);
           ++npvB;
-          if (kn >= 0 && kn <= tB) {
-            ISSUE_QK(1, sK);
-            umma_commit(bar(S_FULL + 1));
-          }
+        }
+        if (kn >= 0 && TAKES_B(kn)) {
+          ISSUE_QK(1, sK);
+          umma_commit(bar(S_FULL + 1));
         }
         umma_commit(bar(KV_EMPTY + sV));
         if (kn >= 0) umma_commit(bar(KV_EMPTY + sK));
@@ -274,6 +291,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const uint32_t tO = tmem + lane_off + 256 + x * D;
     const int tx = x ? tB : tA;
     const bool px = x ? pB : pA;
+    const int lx = x ? lB : lA, hx = x ? hB : hA;
     if (tx >= 0) {
       const int q0 = tile_orig(p, u, tx);
       const bool row_valid = (q0 + r) < p.n_valid;
@@ -282,7 +300,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       if (px) {
         for (int k = 0; k <= tx && ok; ++k) {
-          if (!ktile_valid(p, u, k)) continue;
+          if (!ktile_valid(p, u, k) || !tile_meets(tile_orig(p, u, k), lx, hx)) continue;
           ok = s2_wait(bar(S_FULL + x), n & 1, abort_flag, status, 4);
           if (!ok) break;
           tc_fence_after();
@@ -291,13 +309,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           for (int j = 0; j < 4; ++j) tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[j * 32]));
           tmem_wait_ld();
 
-          // Masks (the causal triangle of the diagonal tile, padded keys or rows)
-          // only where some row of the warp needs them.
-          const int lim = col_limit(p, u, tx, k, r);
-          if (!__all_sync(0xffffffffu, lim == kTile)) {
+          // Masks (the causal triangle of the diagonal tile, padded keys or rows,
+          // the row's document) only where some row of the warp needs them.
+          int cmin, cmax;
+          row_cols(p, u, tx, k, r, cmin, cmax);
+          if (!__all_sync(0xffffffffu, cmin == 0 && cmax == kTile)) {
 #pragma unroll
             for (int c = 0; c < kTile; ++c)
-              if (c >= lim) s[c] = 0xff800000u;  // -inf
+              if (c < cmin || c >= cmax) s[c] = 0xff800000u;  // -inf
           }
           // Row max as a 4-way tree of 3-input max (short dependency chains), then
           // scaled once (scale > 0 keeps the order).
@@ -412,6 +431,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 
 #undef ISSUE_QK
 #undef ISSUE_PV
+#undef NEXT_K
+#undef TAKES_A
+#undef TAKES_B
 #undef bar
 #undef sQ
 #undef sKV

@@ -45,6 +45,10 @@ struct Plan {
   int kv_ranks;    // max over classes of nseg * ntile (grid of each backward pass = kv_ranks * B * H)
   int hg_fwd, hg_bwd;  // heads interleaved per group of consecutive CTAs (L2 locality)
   float scale_log2;  // log2(e) / sqrt(D)
+  // Packed sequences: per-position document bounds [B, N, 2] = {first position,
+  // one past the last position} of the position's document (original
+  // positions), or null when the sequence is one document.
+  const int* docs;
 };
 
 // Linear CTA index -> (flattened head bh, per-head slot r).  CTAs are issued
@@ -240,6 +244,54 @@ S2_HD void query_range(const Plan& p, const Unit& u, int kt, int qt, int j, int&
 S2_HD int grid_fwd(const Plan& p) { return groups_of(p.B * p.H, p.hg_fwd) * p.hg_fwd * p.ranks; }
 S2_HD int grid_bwd(const Plan& p) { return groups_of(p.B * p.H, p.hg_bwd) * p.hg_bwd * p.kv_ranks; }
 
+// ---------------------------------------------------------------- document mask
+// Packed sequences ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1): key j
+// is visible from query i only if both lie in the same document, for both head
+// classes.  Documents are contiguous runs of original positions, so the keys
+// of i's document form the range [doc_lo(i), doc_hi(i)), and a query tile and
+// a key tile (each a contiguous range of original positions) hold a pair in
+// the same document iff the key tile meets the span of the documents that
+// touch the query tile (and symmetrically).
+
+S2_HD int doc_lo(const Plan& p, int b, int x) { return p.docs[(((long long)b * p.N) + x) * 2]; }
+S2_HD int doc_hi(const Plan& p, int b, int x) { return p.docs[(((long long)b * p.N) + x) * 2 + 1]; }
+
+// Span [lo, hi) of the documents touching the tile of 128 rows starting at
+// original position x0 (everything when there are no documents).
+S2_HD void doc_span(const Plan& p, int b, int x0, int& lo, int& hi) {
+  if (!p.docs) { lo = 0; hi = p.N; return; }
+  lo = doc_lo(p, b, x0);
+  hi = doc_hi(p, b, x0 + kTile - 1);
+}
+
+// The tile of 128 positions starting at x0 meets the span [lo, hi).
+S2_HD bool tile_meets(int x0, int lo, int hi) { return x0 < hi && x0 + kTile > lo; }
+
+// Key columns [cmin, cmax) of key tile k visible from row r of query tile tq:
+// the causal diagonal, padding, and the row's document.
+S2_HD void row_cols(const Plan& p, const Unit& u, int tq, int k, int r, int& cmin, int& cmax) {
+  cmin = 0;
+  cmax = col_limit(p, u, tq, k, r);
+  if (p.docs && cmax > 0) {
+    const int k0 = tile_orig(p, u, k), x = tile_orig(p, u, tq) + r;
+    const int lo = doc_lo(p, u.b, x) - k0, hi = doc_hi(p, u.b, x) - k0;
+    if (lo > cmin) cmin = lo;
+    if (hi < cmax) cmax = hi;
+  }
+}
+
+// Query columns [lo, hi) of query tile qt visible from key row j of key tile
+// kt (the same set as row_cols, seen from the key side).
+S2_HD void key_cols(const Plan& p, const Unit& u, int kt, int qt, int j, int& lo, int& hi) {
+  query_range(p, u, kt, qt, j, lo, hi);
+  if (p.docs && hi > lo) {
+    const int q0 = tile_orig(p, u, qt), y = tile_orig(p, u, kt) + j;
+    const int dl = doc_lo(p, u.b, y) - q0, dh = doc_hi(p, u.b, y) - q0;
+    if (dl > lo) lo = dl;
+    if (dh < hi) hi = dh;
+  }
+}
+
 // Host-side plan construction (validated by the caller).
 inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int variant) {
   Plan p{};
@@ -264,6 +316,7 @@ inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int varian
   p.hg_fwd = 2;
   p.hg_bwd = 1;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
+  p.docs = nullptr;
   return p;
 }
 

@@ -1,6 +1,8 @@
 // s2_kernels.h -- internal launch interface between the C-ABI layer and the
 // kernels (not installed; the public interface is include/s2attn.h).
 #pragma once
+#include <cstdint>
+
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -44,5 +46,8 @@ int launch_bwd(const BwdArgs& a, int stages);
 int report_error(int code, const char* fmt, ...);
 
 int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
+
+// Per-position document bounds [B, N, 2] from per-position document IDs [B, N].
+int launch_doc_bounds(const int32_t* ids, int32_t* bounds, int B, int N, cudaStream_t stream);
 
 }  // namespace s2

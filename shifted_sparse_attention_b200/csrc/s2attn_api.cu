@@ -150,12 +150,13 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 101; }
+int s2attn_version(void) { return 102; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
-int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
-                 int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* docs,
+                    int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                    void* stream) {
   int rc = validate(B, N, H, D, G, n_valid, variant);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse) return fail(S2_ERR_INVALID_ARG, "null pointer argument");
@@ -170,15 +171,42 @@ int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* ls
   s2::FwdArgs a;
   a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmO = &to;
   a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  a.plan.docs = docs;
   a.lse = lse;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_fwd(a), "forward");
 }
 
+int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
+                 int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* stream) {
+  return fwd_impl(q, k, v, o, lse, nullptr, B, N, H, D, G, n_valid, variant, stream);
+}
+
 int s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
                int64_t H, int64_t D, int64_t G, int variant, void* stream) {
   return s2attn_fwd_v(q, k, v, o, lse, B, N, H, D, G, N, variant, stream);
+}
+
+int s2attn_fwd_docs(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* doc_bounds,
+                    int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                    void* stream) {
+  if (!doc_bounds) return fail(S2_ERR_INVALID_ARG, "null doc_bounds (use s2attn_fwd_v without documents)");
+  if (reinterpret_cast<uintptr_t>(doc_bounds) & 7u) return fail(S2_ERR_INVALID_ARG, "doc_bounds must be 8-byte aligned");
+  return fwd_impl(q, k, v, o, lse, doc_bounds, B, N, H, D, G, n_valid, variant, stream);
+}
+
+int s2attn_doc_bounds(const int32_t* doc_ids, int32_t* doc_bounds, int64_t B, int64_t N, void* stream) {
+  if (B < 1 || N < 1) return fail(S2_ERR_SHAPE, "B=%lld and N=%lld must be positive", (long long)B, (long long)N);
+  if (B * N >= (int64_t(1) << 30)) return fail(S2_ERR_UNSUPPORTED, "B*N must be below 2^30");
+  if (!doc_ids || !doc_bounds) return fail(S2_ERR_INVALID_ARG, "null pointer argument");
+  if ((reinterpret_cast<uintptr_t>(doc_ids) & 3u) || (reinterpret_cast<uintptr_t>(doc_bounds) & 7u))
+    return fail(S2_ERR_INVALID_ARG, "doc_ids must be 4-byte and doc_bounds 8-byte aligned");
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  return launch_status(s2::launch_doc_bounds(doc_ids, doc_bounds, (int)B, (int)N, static_cast<cudaStream_t>(stream)),
+                       "document bounds");
 }
 
 // Workspace = [-Delta: B*H*N f32][-lse*log2(e): B*H*N f32], each part starting
@@ -192,10 +220,10 @@ size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
   return 2 * stat_bytes(B, N, H);
 }
 
-int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                        const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D,
-                        int64_t G, int64_t n_valid, int variant, void* workspace, size_t workspace_bytes,
-                        int stages, void* stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, const int32_t* docs, void* dq, void* dk, void* dv, int64_t B, int64_t N,
+                    int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace,
+                    size_t workspace_bytes, int stages, void* stream) {
   if (stages < 1 || stages > S2_BWD_ALL) return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7");
   int rc = validate(B, N, H, D, G, n_valid, variant);
   if (rc) return rc;
@@ -220,6 +248,7 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
   s2::BwdArgs a;
   a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmdO = &tdo; a.tmdK = &tdk; a.tmdV = &tdv; a.tmdQ = &tdq;
   a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  a.plan.docs = docs;
   a.o = o;
   a.dout = dout;
   a.lse = lse;
@@ -229,6 +258,24 @@ int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void*
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");
+}
+
+int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H, int64_t D,
+                        int64_t G, int64_t n_valid, int variant, void* workspace, size_t workspace_bytes,
+                        int stages, void* stream) {
+  return bwd_impl(q, k, v, o, dout, lse, nullptr, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,
+                  workspace_bytes, stages, stream);
+}
+
+int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                    const int32_t* doc_bounds, void* dq, void* dk, void* dv, int64_t B, int64_t N, int64_t H,
+                    int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace, size_t workspace_bytes,
+                    int stages, void* stream) {
+  if (!doc_bounds) return fail(S2_ERR_INVALID_ARG, "null doc_bounds (use s2attn_bwd_stages_v without documents)");
+  if (reinterpret_cast<uintptr_t>(doc_bounds) & 7u) return fail(S2_ERR_INVALID_ARG, "doc_bounds must be 8-byte aligned");
+  return bwd_impl(q, k, v, o, dout, lse, doc_bounds, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,
+                  workspace_bytes, stages, stream);
 }
 
 int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,

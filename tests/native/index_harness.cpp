@@ -64,6 +64,78 @@ int s2h_visit_bwd(int N, int G, int n_valid, int variant, int cls, uint8_t* visi
   return units;
 }
 
+// Traversals under a document mask (docs: per-position bounds [N][2], as the
+// kernels read them), for the forward, the dK/dV pass and the dQ pass:
+// visited[i*N + j] += 1 for every computed pair.  `which`: 0 forward, 1 dK/dV,
+// 2 dQ.  docs == nullptr walks the plain graph.
+int s2h_visit_docs(int N, int G, int n_valid, int variant, int cls, const int32_t* docs, int which,
+                   uint8_t* visited) {
+  s2::Plan p = s2::make_plan(1, N, 2, 128, G, n_valid, variant);
+  p.docs = docs;
+  int units = 0;
+  if (which == 0) {
+    for (int L = 0; L < s2::grid_fwd(p); ++L) {
+      s2::Unit u;
+      if (!s2::decode_unit(p, L, u) || u.h != cls) continue;
+      ++units;
+      for (int x = 0; x < 2; ++x) {
+        if (!u.part[x]) continue;
+        const int q0 = s2::tile_orig(p, u, u.t[x]);
+        int lo, hi;
+        s2::doc_span(p, u.b, q0, lo, hi);
+        for (int k = 0; k <= u.t[x]; ++k) {
+          if (!s2::ktile_valid(p, u, k) || !s2::tile_meets(s2::tile_orig(p, u, k), lo, hi)) continue;
+          const int k0 = s2::tile_orig(p, u, k);
+          for (int r = 0; r < s2::kTile; ++r) {
+            int c0, c1;
+            s2::row_cols(p, u, u.t[x], k, r, c0, c1);
+            for (int c = c0; c < c1; ++c) visited[(size_t)(q0 + r) * N + (k0 + c)] += 1;
+          }
+        }
+      }
+    }
+  } else if (which == 1) {
+    for (int L = 0; L < s2::grid_bwd(p); ++L) {
+      s2::Unit u;
+      if (!s2::decode_kv_unit(p, L, u) || u.h != cls) continue;
+      ++units;
+      if (!u.part[0]) continue;
+      const int kt = u.t[0], k0 = s2::tile_orig(p, u, kt);
+      int lo, hi;
+      s2::doc_span(p, u.b, k0, lo, hi);
+      for (int qt = kt; qt <= u.kmax; ++qt) {
+        if (!s2::ktile_valid(p, u, qt) || !s2::tile_meets(s2::tile_orig(p, u, qt), lo, hi)) continue;
+        const int q0 = s2::tile_orig(p, u, qt);
+        for (int j = 0; j < s2::kTile; ++j) {
+          int a, b;
+          s2::key_cols(p, u, kt, qt, j, a, b);
+          for (int i = a; i < b; ++i) visited[(size_t)(q0 + i) * N + (k0 + j)] += 1;
+        }
+      }
+    }
+  } else {
+    for (int L = 0; L < s2::grid_bwd(p); ++L) {
+      s2::Unit u;
+      if (!s2::decode_q_unit(p, L, u) || u.h != cls) continue;
+      ++units;
+      if (!u.part[0]) continue;
+      const int qt = u.t[0], q0 = s2::tile_orig(p, u, qt);
+      int lo, hi;
+      s2::doc_span(p, u.b, q0, lo, hi);
+      for (int k = 0; k <= qt; ++k) {
+        if (!s2::ktile_valid(p, u, k) || !s2::tile_meets(s2::tile_orig(p, u, k), lo, hi)) continue;
+        const int k0 = s2::tile_orig(p, u, k);
+        for (int r = 0; r < s2::kTile; ++r) {
+          int c0, c1;
+          s2::row_cols(p, u, qt, k, r, c0, c1);
+          for (int c = c0; c < c1; ++c) visited[(size_t)(q0 + r) * N + (k0 + c)] += 1;
+        }
+      }
+    }
+  }
+  return units;
+}
+
 // Grid size and per-class unit counts of a launch.
 void s2h_plan(int B, int N, int H, int G, int n_valid, int variant, int32_t* out) {
   s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);

@@ -33,6 +33,8 @@ def harness(tmp_path_factory):
     L.s2h_visit_bwd.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p]
     L.s2h_visit_bwd.restype = ctypes.c_int
     L.s2h_plan.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p]
+    L.s2h_visit_docs.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    L.s2h_visit_docs.restype = ctypes.c_int
     return L
 
 
@@ -72,6 +74,71 @@ def test_scheduler_dense_causal(harness, N):
             np.testing.assert_array_equal(vis.astype(bool), oracle.adjacency(N, N, nv, 2, 0))
 
 
+def _bounds_of(ids):
+    """Per-position [first, one past last] of each maximal run of equal IDs (reference for the kernels' input)."""
+    N = len(ids)
+    b = np.zeros((N, 2), dtype=np.int32)
+    start = 0
+    for x in range(1, N + 1):
+        if x == N or ids[x] != ids[x - 1]:
+            b[start:x] = (start, x)
+            start = x
+    return b
+
+
+def _doc_layouts(N, G):
+    """Document boundaries inside groups, on original and on shifted group boundaries, short
+    documents spanning several tiles, and one document."""
+    s = G // 2
+    cuts = [
+        [N],
+        [5, N],
+        [G, N],
+        [s, G + s, N],
+        [100, 300, 301, G + s + 7, N],
+        list(range(97, N, 97)) + [N],
+        [1, 2, 3, N - 3, N],
+    ]
+    out = []
+    for c in cuts:
+        c = sorted(set(x for x in c if 0 < x <= N))
+        ids = np.zeros(N, dtype=np.int32)
+        for d, (a, b) in enumerate(zip([0] + c, c)):
+            ids[a:b] = d
+        out.append(ids)
+    return out
+
+
+@pytest.mark.parametrize("N,G", [(512, 256), (1024, 512), (1536, 512), (2048, 1024)])
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_scheduler_under_document_masks_visits_exactly_the_oracle_pairs(harness, N, G, variant):
+    if variant == 2:
+        G = N
+    for ids in _doc_layouts(N, G):
+        bounds = np.ascontiguousarray(_bounds_of(ids))
+        same = ids[:, None] == ids[None, :]
+        for nv in (N, N - 77):
+            for cls in ((0,) if variant == 2 else (0, 1)):
+                A = oracle.adjacency(N, G, nv, variant, cls) & same
+                assert oracle.pair_count_docs(N, G, nv, variant, cls, ids) == A.sum()
+                for which in (0, 1, 2):
+                    vis = np.zeros((N, N), dtype=np.uint8)
+                    harness.s2h_visit_docs(N, G, nv, variant, cls, bounds.ctypes.data, which, vis.ctypes.data)
+                    where = str((N, G, nv, variant, cls, which, ids[::97][:6]))
+                    assert vis.max() <= 1, "a pair was computed twice " + where
+                    np.testing.assert_array_equal(vis.astype(bool), A, err_msg=where)
+
+
+def test_dq_traversal_without_documents(harness):
+    for N, G, variant in ((1024, 512, 0), (1024, 512, 1), (768, 768, 2)):
+        for nv in (N, N - 200):
+            for cls in ((0,) if variant == 2 else (0, 1)):
+                vis = np.zeros((N, N), dtype=np.uint8)
+                harness.s2h_visit_docs(N, G, nv, variant, cls, None, 2, vis.ctypes.data)
+                assert vis.max() <= 1
+                np.testing.assert_array_equal(vis.astype(bool), oracle.adjacency(N, G, nv, variant, cls))
+
+
 def test_grid_sizes_of_the_workloads(harness):
     out = np.zeros(5, dtype=np.int32)
     # long-context workload: 4 unshifted segments of 32 units, 5 strict shifted segments
@@ -102,7 +169,7 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 101
+    assert L.s2attn_version() == 102
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
