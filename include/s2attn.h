@@ -144,6 +144,25 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
                     int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
                     void* workspace, size_t workspace_bytes, int stages, void* stream);
 
+/* Training / inference graph gap ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调"
+ * §3 "稀疏训练与full推理之间的目标偏移", §2.1 diagnostics).  Training normalises
+ * row i's softmax over its S² set S_i, inference over its full causal history
+ * F_i; when the graph switches, every in-group weight is scaled by
+ * Z_s / (Z_s + Z_out).  From two forwards on the same q, k, v -- `variant`
+ * (strict or rolled: lse_s2, o_s2) and S2_DENSE_CAUSAL with the same n_valid
+ * (lse_full, o_full) -- this writes, per row (float32 [B, H, N]):
+ *   rho[b,h,i]  = exp(lse_s2 - lse_full)   (= Z_s / (Z_s + Z_out) for strict),
+ *   dist[b,h,i] = || o_s2[b,i,h,:] - o_full[b,i,h,:] ||_2,
+ * both 0 on padded rows, and per head class c (0: heads [0,H/2), 1: the
+ * shifted heads) and bucket k = floor(log2(l + 1)) of the row's position l
+ * inside its S² segment, stats[c][k][0..3] = {row count, mean rho, min rho,
+ * mean dist} (float32 [2][S2_GAP_BUCKETS][4], deterministic).  Device
+ * pointers; o in the layout of the forward. */
+#define S2_GAP_BUCKETS 32
+int s2attn_graph_gap(const float* lse_s2, const float* lse_full, const void* o_s2, const void* o_full,
+                     int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                     float* rho, float* dist, float* stats, void* stream);
+
 /* Size of the fixed scratch array behind s2attn_bwd_noalloc_v (32 MiB). */
 #define S2_NOALLOC_SCRATCH_BYTES (32u << 20)
 
@@ -184,7 +203,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 102. */
+/* ABI version of this header (major*100 + minor): 103. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

@@ -32,6 +32,7 @@ SIGNATURES = {
     "s2attn_bwd_noalloc_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                               _int, _vp], _int),
     "s2attn_doc_bounds": ([_vp, _vp, _i64, _i64, _vp], _int),
+    "s2attn_graph_gap": ([_fp, _fp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _fp, _fp, _fp, _vp], _int),
     "s2attn_fwd_docs": ([_vp, _vp, _vp, _vp, _fp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_bwd_docs": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                          _int, _vp, _sz, _int, _vp], _int),
@@ -145,6 +146,32 @@ def s2attn_bwd_docs(q, k, v, o, dout, lse, doc_bounds, dq, dk, dv, B, N, H, D, G
     return lib().s2attn_bwd_docs(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(doc_bounds),
                                  _ptr(dq), _ptr(dk), _ptr(dv), B, N, H, D, G, n_valid, variant, _ptr(workspace),
                                  workspace_bytes, stages, _stream(stream))
+
+
+def s2attn_graph_gap(lse_s2, lse_full, o_s2, o_full, B, N, H, D, G, n_valid, variant, rho, dist, stats,
+                     stream=None) -> int:
+    return lib().s2attn_graph_gap(_ptr(lse_s2), _ptr(lse_full), _ptr(o_s2), _ptr(o_full), B, N, H, D, G, n_valid,
+                                  variant, _ptr(rho), _ptr(dist), _ptr(stats), _stream(stream))
+
+
+S2_GAP_BUCKETS = 32
+
+
+def graph_gap(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None, stream=None):
+    """Training / inference graph gap of one attention layer: runs the S² and the
+    dense causal forward on the same inputs and returns (rho, dist, stats): per
+    row rho = exp(lse_S2 - lse_full) and dist = ||o_S2 - o_full||_2 ([B, H, N]
+    float32), and per head class and segment-position bucket the row count,
+    mean rho, min rho and mean dist ([2, S2_GAP_BUCKETS, 4])."""
+    B, N, H, D = _shape(q)
+    nv = N if n_valid is None else int(n_valid)
+    o_s, l_s = forward(q, k, v, G, variant, nv, stream=stream)
+    o_f, l_f = forward(q, k, v, N, DENSE_CAUSAL, nv, stream=stream)
+    rho = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    dist = torch.empty_like(rho)
+    stats = torch.empty((2, S2_GAP_BUCKETS, 4), dtype=torch.float32, device=q.device)
+    _check(s2attn_graph_gap(l_s, l_f, o_s, o_f, B, N, H, D, G, nv, variant, rho, dist, stats, stream))
+    return rho, dist, stats
 
 
 def s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, out, stream=None) -> int:

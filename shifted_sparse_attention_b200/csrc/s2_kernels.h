@@ -47,6 +47,12 @@ int report_error(int code, const char* fmt, ...);
 
 int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
 
+// Training / inference graph gap: per-row rho and output shift, per (head
+// class, bucket) statistics float32 [2][kGapBuckets][4].
+constexpr int kGapBuckets = 32;
+int launch_graph_gap(const Plan& p, const float* lse_s, const float* lse_f, const void* o_s, const void* o_f,
+                     float* rho, float* dist, float* stats, cudaStream_t stream);
+
 // Per-position document bounds [B, N, 2] from per-position document IDs [B, N].
 int launch_doc_bounds(const int32_t* ids, int32_t* bounds, int B, int N, cudaStream_t stream);
 

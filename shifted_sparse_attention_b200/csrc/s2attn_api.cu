@@ -150,7 +150,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 102; }
+int s2attn_version(void) { return 103; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -194,6 +194,26 @@ int s2attn_fwd_docs(const void* q, const void* k, const void* v, void* o, float*
   if (!doc_bounds) return fail(S2_ERR_INVALID_ARG, "null doc_bounds (use s2attn_fwd_v without documents)");
   if (reinterpret_cast<uintptr_t>(doc_bounds) & 7u) return fail(S2_ERR_INVALID_ARG, "doc_bounds must be 8-byte aligned");
   return fwd_impl(q, k, v, o, lse, doc_bounds, B, N, H, D, G, n_valid, variant, stream);
+}
+
+int s2attn_graph_gap(const float* lse_s2, const float* lse_full, const void* o_s2, const void* o_full, int64_t B,
+                     int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, float* rho, float* dist,
+                     float* stats, void* stream) {
+  int rc = validate(B, N, H, D, G, n_valid, variant);
+  if (rc) return rc;
+  if (variant == S2_DENSE_CAUSAL) return fail(S2_ERR_INVALID_ARG, "variant must be the S² graph (strict or rolled)");
+  if (!lse_s2 || !lse_full || !o_s2 || !o_full || !rho || !dist || !stats)
+    return fail(S2_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(o_s2) || !aligned16(o_full) || (reinterpret_cast<uintptr_t>(lse_s2) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse_full) & 3u) || (reinterpret_cast<uintptr_t>(rho) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dist) & 3u) || (reinterpret_cast<uintptr_t>(stats) & 3u))
+    return fail(S2_ERR_INVALID_ARG, "misaligned pointer");
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  const s2::Plan p = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  return launch_status(
+      s2::launch_graph_gap(p, lse_s2, lse_full, o_s2, o_full, rho, dist, stats, static_cast<cudaStream_t>(stream)),
+      "graph gap");
 }
 
 int s2attn_doc_bounds(const int32_t* doc_ids, int32_t* doc_bounds, int64_t B, int64_t N, void* stream) {
