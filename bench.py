@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--doc-len", type=int, default=0,
                     help="pack documents of this many tokens (document mask); reports exact-pair TFLOP/s")
+    ap.add_argument("--rope", action="store_true",
+                    help="start each step with the RoPE prologue (original positions, interpolation 1/4)")
     return ap.parse_args()
 
 
@@ -307,22 +309,34 @@ def run_ours(args, rank, world, local_rank):
             raise SystemExit("--doc-len supports the strict and dense variants without padding")
         ids = (torch.arange(N, device=dev, dtype=torch.int32) // args.doc_len).expand(B, N).contiguous()
         docs = s2.doc_bounds(ids)
+    # RoPE prologue: rotate the step's raw Q/K at original positions (restarting per
+    # packed document) with interpolation factor 1/4 into separate buffers
+    q_in, k_in = q, k
+    positions = None
+    if args.rope:
+        q_in, k_in = torch.empty_like(q), torch.empty_like(k)
+        if args.doc_len:
+            positions = (torch.arange(N, device=dev, dtype=torch.int32) % args.doc_len).expand(B, N).contiguous()
 
     def step(ev=None):
+        if args.rope:
+            if ev is not None:
+                ev[5].record(stream)
+            s2.rope(q, k, positions, scale=0.25, out=(q_in, k_in))
         if ev is not None:
             ev[0].record(stream)
-        s2.forward(q, k, v, G, variant, nv, out=o, lse=lse, docs=docs)
+        s2.forward(q_in, k_in, v, G, variant, nv, out=o, lse=lse, docs=docs)
         if ev is not None:
             ev[1].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE,
+        s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE,
                     docs=docs)
         if ev is not None:
             ev[2].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DKDV,
+        s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DKDV,
                     docs=docs)
         if ev is not None:
             ev[3].record(stream)
-        s2.backward(q, k, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ,
+        s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ,
                     docs=docs)
         if ev is not None:
             ev[4].record(stream)
@@ -332,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     s2.check_status()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -351,7 +365,8 @@ def run_ours(args, rank, world, local_rank):
     s2.check_status()
     ms = start.elapsed_time(end)
     per = {name: sum(e[a].elapsed_time(e[b]) for e in evs) / args.steps
-           for name, a, b in (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_dkdv", 2, 3), ("bwd_dq", 3, 4))}
+           for name, a, b in (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_dkdv", 2, 3), ("bwd_dq", 3, 4))
+           + ((("rope", 5, 0),) if args.rope else ())}
     clocks = clk.summary()
 
     # e2e: the same step through the public API from pinned host buffers, copies included
@@ -448,10 +463,19 @@ def run_ours(args, rank, world, local_rank):
         "exact_pair_tflops": (world * pairs * 14 * D / (ms_step * 1e-3) / 1e12) if pairs else None,
         "clocks": clocks,
         "e2e": e2e,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": (5 if args.rope else 4) * args.steps,
         "roofline": roof,
         "cpu_baseline": cpu,
     }
+    if args.rope:
+        # HBM-bound prologue: reads and writes Q and K once (plus the positions)
+        rope_bytes = 2 * 2 * q.numel() * q.element_size() + (positions.numel() * 4 if positions is not None else 0)
+        ach = rope_bytes / (per["rope"] * 1e-3) / 1e9
+        line["config"]["rope"] = {"scale": 0.25, "base": 10000.0,
+                                  "positions": "restart per document" if positions is not None else "0..N-1"}
+        line["rope_roofline"] = {"bound": "hbm", "kernel": "s2_rope_kernel", "achieved": ach, "peak": pk["hbm_gbs"],
+                                 "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "algorithmic_bytes_per_launch": rope_bytes,
+                                 "avg_launch_ms": per["rope"], "traffic": _traffic("s2_rope_kernel", "s2_rope.cu")}
     print(json.dumps(line), flush=True)
 
 

@@ -144,6 +144,21 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
                     int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
                     void* workspace, size_t workspace_bytes, int stages, void* stream);
 
+/* Rotary position prologue ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,
+ * "RoPE使用原始位置"): Q and K are rotated at each token's ORIGINAL position
+ * ID, never its index inside a group, with position interpolation p -> p·scale
+ * (scale = L0/L1 when extending a context of L0 tokens to L1).  Pairing:
+ * coordinate k with k + D/2 (the Llama convention), angle
+ * a_k = (p·scale)·base^(-2k/D):
+ *   x'[k] = x[k] cos a_k - x[k+D/2] sin a_k,  x'[k+D/2] = x[k+D/2] cos a_k + x[k] sin a_k.
+ * q, k, q_out, k_out: bf16 [B, N, H, D], device, 16-byte aligned; q_out / k_out
+ * may equal q / k (in place).  positions: int32 [B, N] original position IDs
+ * (e.g. restarting per packed document), or NULL for 0..N-1.  D in {64, 128}.
+ * Angles are formed in double precision (they reach 10^5 rad); the rotation
+ * is done in float and rounded to bf16. */
+int s2attn_rope(const void* q, const void* k, void* q_out, void* k_out, const int32_t* positions,
+                int64_t B, int64_t N, int64_t H, int64_t D, double base, double scale, void* stream);
+
 /* Training / inference graph gap ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调"
  * §3 "稀疏训练与full推理之间的目标偏移", §2.1 diagnostics).  Training normalises
  * row i's softmax over its S² set S_i, inference over its full causal history
@@ -203,7 +218,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 103. */
+/* ABI version of this header (major*100 + minor): 104. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

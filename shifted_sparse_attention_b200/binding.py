@@ -32,6 +32,8 @@ SIGNATURES = {
     "s2attn_bwd_noalloc_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                               _int, _vp], _int),
     "s2attn_doc_bounds": ([_vp, _vp, _i64, _i64, _vp], _int),
+    "s2attn_rope": ([_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_double, _vp],
+                    _int),
     "s2attn_graph_gap": ([_fp, _fp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _fp, _fp, _fp, _vp], _int),
     "s2attn_fwd_docs": ([_vp, _vp, _vp, _vp, _fp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_bwd_docs": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
@@ -152,6 +154,33 @@ def s2attn_graph_gap(lse_s2, lse_full, o_s2, o_full, B, N, H, D, G, n_valid, var
                      stream=None) -> int:
     return lib().s2attn_graph_gap(_ptr(lse_s2), _ptr(lse_full), _ptr(o_s2), _ptr(o_full), B, N, H, D, G, n_valid,
                                   variant, _ptr(rho), _ptr(dist), _ptr(stats), _stream(stream))
+
+
+def s2attn_rope(q, k, q_out, k_out, positions, B, N, H, D, base, scale, stream=None) -> int:
+    return lib().s2attn_rope(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), _ptr(positions), B, N, H, D, float(base),
+                             float(scale), _stream(stream))
+
+
+def rope(q, k, positions=None, base: float = 10000.0, scale: float = 1.0, inplace: bool = False, out=None,
+         stream=None):
+    """Rotary position prologue on original positions (see include/s2attn.h); returns (q', k').
+    ``out``: optional preallocated (q_out, k_out); ``inplace`` rotates q and k themselves."""
+    B, N, H, D = _shape(q)
+    if _shape(k) != (B, N, H, D):
+        raise ValueError("q and k must have the same shape")
+    if positions is not None and (positions.shape != (B, N) or positions.dtype != torch.int32 or not positions.is_cuda
+                                  or not positions.is_contiguous()):
+        raise ValueError("positions must be a contiguous CUDA int32 tensor [B, N]")
+    if inplace:
+        qo, ko = q, k
+    elif out is not None:
+        qo, ko = out
+        if _shape(qo) != (B, N, H, D) or _shape(ko) != (B, N, H, D):
+            raise ValueError("out tensors must match q")
+    else:
+        qo, ko = torch.empty_like(q), torch.empty_like(k)
+    _check(s2attn_rope(q, k, qo, ko, positions, B, N, H, D, base, scale, stream))
+    return qo, ko
 
 
 S2_GAP_BUCKETS = 32

@@ -53,6 +53,10 @@ constexpr int kGapBuckets = 32;
 int launch_graph_gap(const Plan& p, const float* lse_s, const float* lse_f, const void* o_s, const void* o_f,
                      float* rho, float* dist, float* stats, cudaStream_t stream);
 
+// Rotary position prologue on original positions (positions: int32 [B, N] or null = 0..N-1).
+int launch_rope(const void* q, const void* k, void* q_out, void* k_out, const int* positions, int B, int N, int H,
+                int D, double base, double scale, cudaStream_t stream);
+
 // Per-position document bounds [B, N, 2] from per-position document IDs [B, N].
 int launch_doc_bounds(const int32_t* ids, int32_t* bounds, int B, int N, cudaStream_t stream);
 

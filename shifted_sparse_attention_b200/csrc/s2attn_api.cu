@@ -150,7 +150,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 103; }
+int s2attn_version(void) { return 104; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -214,6 +214,24 @@ int s2attn_graph_gap(const float* lse_s2, const float* lse_full, const void* o_s
   return launch_status(
       s2::launch_graph_gap(p, lse_s2, lse_full, o_s2, o_full, rho, dist, stats, static_cast<cudaStream_t>(stream)),
       "graph gap");
+}
+
+int s2attn_rope(const void* q, const void* k, void* q_out, void* k_out, const int32_t* positions, int64_t B,
+                int64_t N, int64_t H, int64_t D, double base, double scale, void* stream) {
+  if (B < 1 || N < 1 || H < 1) return fail(S2_ERR_SHAPE, "B, N, H must be positive");
+  if (D != 64 && D != 128) return fail(S2_ERR_UNSUPPORTED, "D=%lld: the prologue supports D in {64, 128}", (long long)D);
+  if (B * N >= (int64_t(1) << 31) || B * N * H * D >= (int64_t(1) << 62)) return fail(S2_ERR_UNSUPPORTED, "too large");
+  if (!(base > 1.0) || !(scale > 0.0)) return fail(S2_ERR_INVALID_ARG, "base must be > 1 and scale > 0");
+  if (!q || !k || !q_out || !k_out) return fail(S2_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_out) || !aligned16(k_out) ||
+      (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return fail(S2_ERR_INVALID_ARG, "q, k, q_out, k_out must be 16-byte aligned (positions 4-byte)");
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  return launch_status(s2::launch_rope(q, k, q_out, k_out, positions, (int)B, (int)N, (int)H, (int)D, base, scale,
+                                       static_cast<cudaStream_t>(stream)),
+                       "rope");
 }
 
 int s2attn_doc_bounds(const int32_t* doc_ids, int32_t* doc_bounds, int64_t B, int64_t N, void* stream) {

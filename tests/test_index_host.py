@@ -169,7 +169,7 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 103
+    assert L.s2attn_version() == 104
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
@@ -209,3 +209,22 @@ def test_tensor_api_refuses_cpu_tensors(abi):
     q = torch.zeros(1, 1024, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         abi.forward(q, q, q, 256)
+
+
+def test_rope_host_validation(abi):
+    L = abi.lib()
+    fake = 1 << 20
+    rc = L.s2attn_rope(fake, fake, fake, fake, None, 1, 16, 2, 96, 10000.0, 1.0, None)
+    assert rc == abi.S2_ERR_UNSUPPORTED  # D outside {64, 128}
+    rc = L.s2attn_rope(fake, fake, fake, fake, None, 1, 16, 2, 128, 1.0, 1.0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # base must exceed 1
+    rc = L.s2attn_rope(fake, fake, fake, fake, None, 1, 16, 2, 128, 10000.0, 0.0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # scale must be positive
+    rc = L.s2attn_rope(fake, None, fake, fake, None, 1, 16, 2, 128, 10000.0, 1.0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG
+    rc = L.s2attn_rope(fake, fake, fake + 4, fake, None, 1, 16, 2, 128, 10000.0, 1.0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # misaligned output
+    rc = L.s2attn_rope(fake, fake, fake, fake, fake + 2, 1, 16, 2, 128, 10000.0, 1.0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # misaligned positions
+    rc = L.s2attn_rope(fake, fake, fake, fake, None, 0, 16, 2, 128, 10000.0, 1.0, None)
+    assert rc == abi.S2_ERR_SHAPE
