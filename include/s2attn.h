@@ -159,6 +159,64 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
 int s2attn_rope(const void* q, const void* k, void* q_out, void* k_out, const int32_t* positions,
                 int64_t B, int64_t N, int64_t H, int64_t D, double base, double scale, void* stream);
 
+/* Sequence parallelism ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,
+ * "Sequence Parallel通信"): the sequence of N = world·L positions is cut into
+ * G-aligned shards, rank r holding original positions [rL, rL + L).  Group
+ * boundaries of the unshifted heads then coincide with shard boundaries; the
+ * shifted heads' group straddling a boundary needs, on rank r, the s = G/2
+ * K/V rows [rL - s, rL) of rank r - 1 (the halo), and returns their partial
+ * gradients to it.  Exchanging only this halo (never rolling inside a shard)
+ * keeps the multi-rank graph identical to the single-GPU graph.
+ *
+ * Layout: every tensor of a rank lives in an EXTENDED buffer of s + L rows,
+ * [B, s + L, H, D] bf16 (lse [B, H, s + L] fp32), whose rows [0, s) are the
+ * halo and rows [s, s + L) the shard.  Halo rows of q, dout are never read;
+ * those of o, lse, dq are overwritten with zeros (-inf for lse); those of
+ * dk, dv receive the shard's partial gradients of the halo keys.
+ *
+ * One forward or backward step of a rank:
+ *   1. s2attn_sp_halo_pack(k, v, msg, ..., S2_SP_KV): the shard's last s rows
+ *      of the shifted heads -> msg (s2attn_sp_halo_bytes bytes); send msg to
+ *      rank r + 1 (ROLLED: to (r + 1) mod world; STRICT: the last rank sends
+ *      nothing); receive into msg' from rank r - 1 and
+ *      s2attn_sp_halo_unpack(msg', k, v, ..., S2_SP_KV) into the halo rows.
+ *      (Rank 0 of a STRICT sequence receives nothing; its halo is ignored.)
+ *   2. s2attn_sp_fwd / s2attn_sp_bwd on the extended buffers.
+ *   3. After the backward: s2attn_sp_halo_pack(dk, dv, msg, ..., S2_SP_GRAD)
+ *      sends the halo rows' gradients back to the rank the halo came from,
+ *      which adds them with s2attn_sp_halo_unpack(..., S2_SP_GRAD) onto its
+ *      last s rows (fp32 sum, one rounding to bf16).
+ * With world = 1, ROLLED sends to itself and STRICT sends nothing; both then
+ * equal the single-GPU calls.  O, lse and dq of every shard row are bitwise
+ * those of the single-GPU call on the whole sequence (same tiles, same order);
+ * dk, dv of the s rows in front of each boundary differ by the extra rounding
+ * of the two partial sums.
+ *
+ * Arguments: L = rows of the shard (a multiple of G); n_valid = valid rows of
+ * the shard (L except on a padded last rank; ROLLED needs n_valid = L);
+ * variant S2_STRICT or S2_ROLLED (S2_DENSE_CAUSAL does not shard this way:
+ * S2_ERR_UNSUPPORTED); workspace: s2attn_bwd_workspace_size(B, G/2 + L, H, D)
+ * bytes.  The messages are [2][B][s][H/2][D] bf16: V_KV = 2·B·(H/2)·s·D·2
+ * bytes per direction, the pages' volume. */
+enum { S2_SP_KV = 0, S2_SP_GRAD = 1 };
+
+int s2attn_sp_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t L,
+                  int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, int rank, int world,
+                  void* stream);
+
+int s2attn_sp_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t L, int64_t H,
+                  int64_t D, int64_t G, int64_t n_valid, int variant, int rank, int world,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+size_t s2attn_sp_halo_bytes(int64_t B, int64_t H, int64_t D, int64_t G);
+
+int s2attn_sp_halo_pack(const void* a, const void* b, void* msg, int64_t B, int64_t L, int64_t H,
+                        int64_t D, int64_t G, int part, void* stream);
+
+int s2attn_sp_halo_unpack(const void* msg, void* a, void* b, int64_t B, int64_t L, int64_t H,
+                          int64_t D, int64_t G, int part, void* stream);
+
 /* Training / inference graph gap ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调"
  * §3 "稀疏训练与full推理之间的目标偏移", §2.1 diagnostics).  Training normalises
  * row i's softmax over its S² set S_i, inference over its full causal history
@@ -218,7 +276,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 104. */
+/* ABI version of this header (major*100 + minor): 105. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

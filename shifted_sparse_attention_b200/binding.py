@@ -38,6 +38,12 @@ SIGNATURES = {
     "s2attn_fwd_docs": ([_vp, _vp, _vp, _vp, _fp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_bwd_docs": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
                          _int, _vp, _sz, _int, _vp], _int),
+    "s2attn_sp_fwd": ([_vp, _vp, _vp, _vp, _fp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int, _int, _vp], _int),
+    "s2attn_sp_bwd": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int,
+                       _int, _vp, _sz, _vp], _int),
+    "s2attn_sp_halo_bytes": ([_i64, _i64, _i64, _i64], _sz),
+    "s2attn_sp_halo_pack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
+    "s2attn_sp_halo_unpack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
@@ -181,6 +187,33 @@ def rope(q, k, positions=None, base: float = 10000.0, scale: float = 1.0, inplac
         qo, ko = torch.empty_like(q), torch.empty_like(k)
     _check(s2attn_rope(q, k, qo, ko, positions, B, N, H, D, base, scale, stream))
     return qo, ko
+
+
+S2_SP_KV, S2_SP_GRAD = 0, 1
+
+
+def s2attn_sp_fwd(q, k, v, o, lse, B, L, H, D, G, n_valid, variant, rank, world, stream=None) -> int:
+    return lib().s2attn_sp_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, L, H, D, G, n_valid, variant, rank,
+                               world, _stream(stream))
+
+
+def s2attn_sp_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, L, H, D, G, n_valid, variant, rank, world, workspace,
+                  workspace_bytes, stream=None) -> int:
+    return lib().s2attn_sp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                               _ptr(dv), B, L, H, D, G, n_valid, variant, rank, world, _ptr(workspace),
+                               workspace_bytes, _stream(stream))
+
+
+def s2attn_sp_halo_bytes(B, H, D, G) -> int:
+    return int(lib().s2attn_sp_halo_bytes(B, H, D, G))
+
+
+def s2attn_sp_halo_pack(a, b, msg, B, L, H, D, G, part, stream=None) -> int:
+    return lib().s2attn_sp_halo_pack(_ptr(a), _ptr(b), _ptr(msg), B, L, H, D, G, part, _stream(stream))
+
+
+def s2attn_sp_halo_unpack(msg, a, b, B, L, H, D, G, part, stream=None) -> int:
+    return lib().s2attn_sp_halo_unpack(_ptr(msg), _ptr(a), _ptr(b), B, L, H, D, G, part, _stream(stream))
 
 
 S2_GAP_BUCKETS = 32

@@ -16,7 +16,7 @@ namespace s2 {
 
 // One CTA per work unit of a head of class `cls`; thread = one row of the
 // unit's two query tiles.
-__global__ void __launch_bounds__(256) s2_adjacency_kernel(const Plan p, int cls, int format,
+__global__ void __launch_bounds__(256) s2_adjacency_kernel(const __grid_constant__ Plan p, int cls, int format,
                                                            uint32_t* __restrict__ bits,
                                                            int* __restrict__ intervals) {
   Unit u;

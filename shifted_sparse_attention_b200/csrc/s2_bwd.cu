@@ -51,7 +51,7 @@ constexpr int kChunkBytes = kTile * 64 * 2;  // 128 rows x 64 bf16: one 128-byte
 // meets the span [lo, hi) of the documents touching the key tile, or -1.
 __device__ __forceinline__ int next_q(const Plan& p, const Unit& u, int qt, int lo, int hi) {
   for (int j = qt + 1; j <= u.kmax; ++j)
-    if (ktile_valid(p, u, j) && tile_meets(tile_orig(p, u, j), lo, hi)) return j;
+    if (qtile_valid(p, u, j) && tile_meets(tile_orig(p, u, j), lo, hi)) return j;
   return -1;
 }
 
@@ -103,7 +103,8 @@ template <int D>
 __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restrict__ o,
                                                    const __nv_bfloat16* __restrict__ dout,
                                                    const float* __restrict__ lse, float* __restrict__ delta,
-                                                   float* __restrict__ lse2, int B, int N, int H, int n_valid) {
+                                                   float* __restrict__ lse2, int B, int N, int H, int q_begin,
+                                                   int n_valid) {
   constexpr int kTpr = D / 8;
   constexpr int kRowsPerBlock = 256 / kTpr;
   const long long row = (long long)blockIdx.x * kRowsPerBlock + threadIdx.x / kTpr;
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restric
     const long long bi = row / H;
     const int i = (int)(bi % N), b = (int)(bi / N);
     const size_t at = ((size_t)b * H + h) * N + i;
-    const bool valid = i < n_valid;
+    const bool valid = i >= q_begin && i < n_valid;
     delta[at] = valid ? -acc : 0.f;
     lse2[at] = valid ? -lse[at] * 1.4426950408889634f : -INFINITY;
   }
@@ -191,7 +192,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                       const Plan p, const float* __restrict__ delta, const float* __restrict__ lse2,
+                       const __grid_constant__ Plan p, const float* __restrict__ delta,
+                       const float* __restrict__ lse2,
                        int* __restrict__ status) {
   using namespace bwd;
   using namespace dkdv;
@@ -208,9 +210,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   }
   const int kt = u.t[0];
   const int k0 = tile_orig(p, u, kt);
-  const bool kvalid = u.part[0];
   int lK, hK;  // span of the documents touching the key tile
   doc_span(p, u.b, k0, lK, hK);
+  // first query tile: the diagonal, unless it lies in a sequence-parallel halo
+  // (rows that are keys only); a key tile no query reaches gets dK = dV = 0
+  const int q_first = !u.part[0] ? -1 : qtile_valid(p, u, kt) ? kt : next_q(p, u, kt, lK, hK);
+  const bool kvalid = q_first >= 0;
 
   uint8_t* smem = smem_kv;
   const uint32_t sb = smem_u32(smem);
@@ -266,7 +271,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
       int n = 0;
       bool ok = true;
-      for (int qt = kt; ok && qt >= 0; qt = next_q(p, u, qt, lK, hK)) {
+      for (int qt = q_first; ok && qt >= 0; qt = next_q(p, u, qt, lK, hK)) {
         const int q0 = tile_orig(p, u, qt);
         const int sq = n % kQSlots, so = n % kOSlots;
         if (n >= kQSlots) ok = s2_wait(bar(Q_EMPTY + sq), ((n / kQSlots) - 1) & 1, abort_flag, status, 8);
@@ -311,8 +316,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       }
       int n = 0;
       if (ok) ok = s2_wait(bar(O_FULL + 0), 0, abort_flag, status, 16);
-      int qn = next_q(p, u, kt, lK, hK);
-      for (int qt = kt; ok && qt >= 0;) {
+      int qn = next_q(p, u, q_first, lK, hK);
+      for (int qt = q_first; ok && qt >= 0;) {
         const int sq = n % kQSlots, sd = n % kOSlots;
         const uint64_t oq = (uint64_t)sq * kSlotStep, od = (uint64_t)sd * kSlotStep;
         // dP^T(n) -> R2 (dO(n) has landed)
@@ -416,7 +421,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         mbar_arrive(bar(P_READY));
         return true;
       };
-      int qt = kt;
+      int qt = q_first;
       ok = p_step(0, qt);
       while (ok && qt >= 0) {
         const int sd = n % kOSlots;
@@ -531,7 +536,8 @@ template <int D>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     s2_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                     const __grid_constant__ CUtensorMap tmdQ, const Plan p, const float* __restrict__ delta,
+                     const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ Plan p,
+                     const float* __restrict__ delta,
                      const float* __restrict__ lse2, int* __restrict__ status) {
   using namespace bwd;
   using namespace dqp;
@@ -810,7 +816,7 @@ int launch_bwd_impl(const BwdArgs& a, int stages) {
     constexpr int kRowsPerBlock = 256 / (D / 8);
     s2_bwd_pre<D><<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, a.stream>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.delta, a.lse2,
-        p.B, p.N, p.H, p.n_valid);
+        p.B, p.N, p.H, p.q_begin, p.n_valid);
     e = cudaGetLastError();
     if (e != cudaSuccess) return (int)e;
   }

@@ -67,27 +67,37 @@ struct Layout {
 
 // Query tile x (its index tx, whether it holds a valid row px, and the span
 // [lo, hi) of the documents touching it) takes part at key tile k.
+// Without documents (kDocs false) the span test is skipped outright: it costs
+// the single MMA-issuing thread a tile-origin computation per key tile.
+template <bool kDocs>
 __device__ __forceinline__ bool takes(const Plan& p, const Unit& u, bool px, int tx, int lo, int hi, int k) {
-  return px && k <= tx && tile_meets(tile_orig(p, u, k), lo, hi);
+  if constexpr (kDocs) return px && k <= tx && tile_meets(tile_orig(p, u, k), lo, hi);
+  return px && k <= tx;
 }
 
 // Smallest key tile > k that holds a valid key and that one of the unit's two
 // query tiles takes part at, or -1.
+template <bool kDocs>
 __device__ __forceinline__ int next_k(const Plan& p, const Unit& u, int k, bool pA, int tA, int lA, int hA, bool pB,
                                       int tB, int lB, int hB) {
   for (int j = k + 1; j <= u.kmax; ++j)
-    if (ktile_valid(p, u, j) && (takes(p, u, pA, tA, lA, hA, j) || takes(p, u, pB, tB, lB, hB, j))) return j;
+    if (ktile_valid(p, u, j) &&
+        (takes<kDocs>(p, u, pA, tA, lA, hA, j) || takes<kDocs>(p, u, pB, tB, lB, hB, j)))
+      return j;
   return -1;
 }
 
 }  // namespace fwd
 
-template <int D>
+// kDocs: a document mask is present (p.docs != nullptr).  Without it the
+// document tests fold away at compile time.
+template <int D, bool kDocs>
 __global__ void __launch_bounds__(fwd::kThreads, 1)
     s2_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                  const Plan p, float* __restrict__ lse, int* __restrict__ status) {
+                  const __grid_constant__ Plan plan, float* __restrict__ lse, int* __restrict__ status) {
   using namespace fwd;
+  const Plan& p = plan;
   using L = Layout<D>;
   constexpr int kChunks = D / 64;
 
@@ -99,11 +109,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
   const bool pA = u.part[0], pB = u.part[1];
   // spans of the documents touching each query tile (everything without documents)
   int lA = 0, hA = p.N, lB = 0, hB = p.N;
-  if (pA) doc_span(p, u.b, tile_orig(p, u, tA), lA, hA);
-  if (pB) doc_span(p, u.b, tile_orig(p, u, tB), lB, hB);
-#define NEXT_K(k) next_k(p, u, (k), pA, tA, lA, hA, pB, tB, lB, hB)
-#define TAKES_A(k) takes(p, u, pA, tA, lA, hA, (k))
-#define TAKES_B(k) takes(p, u, pB, tB, lB, hB, (k))
+  if (kDocs && pA) doc_span(p, u.b, tile_orig(p, u, tA), lA, hA);
+  if (kDocs && pB) doc_span(p, u.b, tile_orig(p, u, tB), lB, hB);
+#define NEXT_K(k) next_k<kDocs>(p, u, (k), pA, tA, lA, hA, pB, tB, lB, hB)
+#define TAKES_A(k) takes<kDocs>(p, u, pA, tA, lA, hA, (k))
+#define TAKES_B(k) takes<kDocs>(p, u, pB, tB, lB, hB, (k))
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -300,7 +310,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       bool ok = true;
       if (px) {
         for (int k = 0; k <= tx && ok; ++k) {
-          if (!ktile_valid(p, u, k) || !tile_meets(tile_orig(p, u, k), lx, hx)) continue;
+          if (!ktile_valid(p, u, k) || (kDocs && !tile_meets(tile_orig(p, u, k), lx, hx))) continue;
           ok = s2_wait(bar(S_FULL + x), n & 1, abort_flag, status, 4);
           if (!ok) break;
           tc_fence_after();
@@ -311,8 +321,11 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 
           // Masks (the causal triangle of the diagonal tile, padded keys or rows,
           // the row's document) only where some row of the warp needs them.
-          int cmin, cmax;
-          row_cols(p, u, tx, k, r, cmin, cmax);
+          int cmin = 0, cmax;
+          if constexpr (kDocs)
+            row_cols(p, u, tx, k, r, cmin, cmax);
+          else
+            cmax = col_limit(p, u, tx, k, r);
           if (!__all_sync(0xffffffffu, cmin == 0 && cmax == kTile)) {
 #pragma unroll
             for (int c = 0; c < kTile; ++c)
@@ -438,21 +451,23 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #undef sQ
 #undef sKV
 
-template <int D>
+template <int D, bool kDocs>
 int launch_fwd_impl(const FwdArgs& a) {
   using L = fwd::Layout<D>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(s2_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+  cudaError_t e =
+      cudaFuncSetAttribute(s2_fwd_kernel<D, kDocs>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
   if (e != cudaSuccess) return (int)e;
   const int grid = grid_fwd(a.plan);
-  s2_fwd_kernel<D><<<grid, fwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmO, a.plan,
-                                                                 a.lse, a.status);
+  s2_fwd_kernel<D, kDocs><<<grid, fwd::kThreads, L::kAlloc, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmO, a.plan,
+                                                                        a.lse, a.status);
   return (int)cudaGetLastError();
 }
 
 int launch_fwd(const FwdArgs& a) {
-  if (a.plan.D == 64) return launch_fwd_impl<64>(a);
-  return launch_fwd_impl<128>(a);
+  const bool docs = a.plan.docs != nullptr;
+  if (a.plan.D == 64) return docs ? launch_fwd_impl<64, true>(a) : launch_fwd_impl<64, false>(a);
+  return docs ? launch_fwd_impl<128, true>(a) : launch_fwd_impl<128, false>(a);
 }
 
 }  // namespace s2

@@ -36,7 +36,7 @@ __device__ __forceinline__ int row_bucket(const Plan& p, int cls, int x) {
   return 31 - __clz(l1);
 }
 
-__global__ void __launch_bounds__(kGapThreads) s2_gap_rows(const Plan p, const float* __restrict__ lse_s,
+__global__ void __launch_bounds__(kGapThreads) s2_gap_rows(const __grid_constant__ Plan p, const float* __restrict__ lse_s,
                                                            const float* __restrict__ lse_f,
                                                            const __nv_bfloat16* __restrict__ o_s,
                                                            const __nv_bfloat16* __restrict__ o_f,
@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(kGapThreads) s2_gap_rows(const Plan p, const f
 }
 
 // stats[(cls * kGapBuckets + k) * 4 + {0,1,2,3}] = {count, mean rho, min rho, mean d}
-__global__ void __launch_bounds__(kGapThreads) s2_gap_stats(const Plan p, const float* __restrict__ rho,
+__global__ void __launch_bounds__(kGapThreads) s2_gap_stats(const __grid_constant__ Plan p, const float* __restrict__ rho,
                                                             const float* __restrict__ dist,
                                                             float* __restrict__ stats) {
   const int cls = blockIdx.x / kGapBuckets, k = blockIdx.x % kGapBuckets;

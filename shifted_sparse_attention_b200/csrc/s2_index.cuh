@@ -21,6 +21,21 @@
 //   ROLLED class 1: virtual index r = rolled position, original = (r + s) mod N.
 // With s a multiple of 128, every 128-row tile of virtual rows is a
 // contiguous range of original positions, so each tile is one TMA box.
+//
+// Segment lattice.  Outside DENSE_CAUSAL, the segments of class c are the
+// intervals [off_c + kG, off_c + (k+1)G) of virtual rows clipped to [0, N):
+// off = {0, s} gives STRICT (the clipped first and last intervals are its
+// short head and tail groups), off = {0, 0} gives class 0 and the rolled
+// coordinates of ROLLED class 1.
+//
+// Sequence parallelism ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,
+// distributed boundaries: the shifted heads exchange a half-group halo with
+// the neighbouring rank): a rank holding the G-aligned shard [rL, rL + L) of a
+// STRICT (or ROLLED) sequence works on an extended buffer of N = s + L rows
+// whose first s rows are the halo, rows [rL - s, rL) of the previous rank.
+// In those coordinates class 0's boundaries sit at s + kG and class 1's at
+// kG, i.e. off = {s, 0}; halo rows are keys only (q_begin = s), and on the
+// first rank of a STRICT sequence they hold no key at all (k_begin = s).
 #pragma once
 #include <cstdint>
 
@@ -44,6 +59,9 @@ struct Plan {
   int ntile[2];    // max tiles per segment, per class
   int kv_ranks;    // max over classes of nseg * ntile (grid of each backward pass = kv_ranks * B * H)
   int hg_fwd, hg_bwd;  // heads interleaved per group of consecutive CTAs (L2 locality)
+  int off[2];      // segment lattice offset per class (see above)
+  int q_begin;     // rows [0, q_begin) are never queries (a sequence-parallel halo)
+  int k_begin;     // rows [0, k_begin) hold no valid key
   float scale_log2;  // log2(e) / sqrt(D)
   // Packed sequences: per-position document bounds [B, N, 2] = {first position,
   // one past the last position} of the position's document (original
@@ -71,32 +89,25 @@ S2_HD int head_class(const Plan& p, int h) {
 
 S2_HD int seg_count(const Plan& p, int cls) {
   if (p.variant == kDenseCausal) return 1;
-  if (cls == 1 && p.variant == kStrict) return p.N / p.G + 1;
-  return p.N / p.G;
+  const int o = p.off[cls];
+  return (o ? 1 : 0) + (p.N - o + p.G - 1) / p.G;
 }
 
 // Virtual range [vbeg, vbeg + len) of segment `seg`.
 S2_HD void seg_bounds(const Plan& p, int cls, int seg, int& vbeg, int& len) {
   if (p.variant == kDenseCausal) { vbeg = 0; len = p.N; return; }
-  if (cls == 1 && p.variant == kStrict) {
-    const int M = p.N / p.G;
-    if (seg == 0) { vbeg = 0; len = p.s; return; }
-    if (seg == M) { vbeg = p.N - p.s; len = p.s; return; }
-    vbeg = p.s + (seg - 1) * p.G; len = p.G; return;
-  }
-  vbeg = seg * p.G; len = p.G;
+  const int o = p.off[cls];
+  if (o && seg == 0) { vbeg = 0; len = o; return; }
+  vbeg = o + (seg - (o ? 1 : 0)) * p.G;
+  len = p.N - vbeg < p.G ? p.N - vbeg : p.G;
 }
 
 // Segment containing virtual row v.
 S2_HD int seg_of(const Plan& p, int cls, int v) {
   if (p.variant == kDenseCausal) return 0;
-  if (cls == 1 && p.variant == kStrict) {
-    if (v < p.s) return 0;
-    const int M = p.N / p.G;
-    if (v >= p.N - p.s) return M;
-    return (v - p.s) / p.G + 1;
-  }
-  return v / p.G;
+  const int o = p.off[cls];
+  if (v < o) return 0;
+  return (v - o) / p.G + (o ? 1 : 0);
 }
 
 S2_HD int orig_of(const Plan& p, int cls, int v) {
@@ -130,6 +141,18 @@ S2_HD int tile_orig(const Plan& p, const Unit& u, int t) {
   return orig_of(p, u.cls, u.vbeg + t * kTile);
 }
 
+// A key tile is processed iff it holds at least one valid key; a query tile
+// iff it holds at least one valid query row.  (n_valid cuts inside a tile;
+// q_begin and k_begin are multiples of the tile.)
+S2_HD bool ktile_valid(const Plan& p, const Unit& u, int k) {
+  const int x0 = tile_orig(p, u, k);
+  return x0 >= p.k_begin && x0 < p.n_valid;
+}
+S2_HD bool qtile_valid(const Plan& p, const Unit& u, int t) {
+  const int x0 = tile_orig(p, u, t);
+  return x0 >= p.q_begin && x0 < p.n_valid;
+}
+
 // Decode a linear work index (longest work first).  Returns false for idle indices.
 S2_HD bool decode_unit(const Plan& p, int L, Unit& u) {
   int bh, r;
@@ -149,15 +172,10 @@ S2_HD bool decode_unit(const Plan& p, int L, Unit& u) {
   u.t[1] = (2 * unit + 1 < u.ntiles) ? 2 * unit + 1 : -1;
   u.kmax = -1;
   for (int x = 0; x < 2; ++x) {
-    u.part[x] = (u.t[x] >= 0) && (tile_orig(p, u, u.t[x]) < p.n_valid);
+    u.part[x] = (u.t[x] >= 0) && qtile_valid(p, u, u.t[x]);
     if (u.part[x]) u.kmax = u.t[x];
   }
   return true;
-}
-
-// A key tile is processed iff it holds at least one valid key.
-S2_HD bool ktile_valid(const Plan& p, const Unit& u, int k) {
-  return tile_orig(p, u, k) < p.n_valid;
 }
 
 // Query tile x takes part at key tile k.
@@ -199,7 +217,7 @@ S2_HD bool decode_kv_unit(const Plan& p, int L, Unit& u) {
   if (kt >= u.ntiles) return false;
   u.t[0] = kt;
   u.t[1] = -1;
-  u.part[0] = tile_orig(p, u, kt) < p.n_valid;
+  u.part[0] = ktile_valid(p, u, kt);
   u.part[1] = false;
   u.kmax = u.ntiles - 1;
   return true;
@@ -225,7 +243,7 @@ S2_HD bool decode_q_unit(const Plan& p, int L, Unit& u) {
   if (qt < 0) return false;
   u.t[0] = qt;
   u.t[1] = -1;
-  u.part[0] = tile_orig(p, u, qt) < p.n_valid;
+  u.part[0] = qtile_valid(p, u, qt);
   u.part[1] = false;
   u.kmax = qt;
   return true;
@@ -292,11 +310,8 @@ S2_HD void key_cols(const Plan& p, const Unit& u, int kt, int qt, int j, int& lo
   }
 }
 
-// Host-side plan construction (validated by the caller).
-inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int variant) {
-  Plan p{};
-  p.B = B; p.N = N; p.H = H; p.D = D; p.G = G; p.s = G / 2;
-  p.n_valid = n_valid; p.variant = variant;
+// Per-class unit and tile counts of a plan whose geometry is set.
+inline void finish_plan(Plan& p) {
   for (int c = 0; c < 2; ++c) {
     p.nseg[c] = seg_count(p, c);
     int maxlen = 0;
@@ -315,8 +330,38 @@ inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int varian
   p.kv_ranks = k0 > k1 ? k0 : k1;
   p.hg_fwd = 2;
   p.hg_bwd = 1;
-  p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
+  p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)p.D));
+}
+
+// Host-side plan construction (validated by the caller).
+inline Plan make_plan(int B, int N, int H, int D, int G, int n_valid, int variant) {
+  Plan p{};
+  p.B = B; p.N = N; p.H = H; p.D = D; p.G = G; p.s = G / 2;
+  p.n_valid = n_valid; p.variant = variant;
+  p.off[0] = 0;
+  p.off[1] = (variant == kStrict) ? p.s : 0;
+  p.q_begin = 0;
+  p.k_begin = 0;
   p.docs = nullptr;
+  finish_plan(p);
+  return p;
+}
+
+// Plan of one sequence-parallel rank over its extended buffer of s + L rows
+// (halo first).  n_valid counts extended rows; first_strict: the rank holds
+// the start of a STRICT sequence, so its halo rows are not keys.
+inline Plan make_plan_sp(int B, int L, int H, int D, int G, int n_valid, bool first_strict) {
+  Plan p{};
+  p.B = B; p.H = H; p.D = D; p.G = G; p.s = G / 2;
+  p.N = p.s + L;
+  p.n_valid = n_valid;
+  p.variant = kStrict;  // plain (unrolled) coordinates in the extended buffer
+  p.off[0] = p.s;
+  p.off[1] = 0;
+  p.q_begin = p.s;
+  p.k_begin = first_strict ? p.s : 0;
+  p.docs = nullptr;
+  finish_plan(p);
   return p;
 }
 

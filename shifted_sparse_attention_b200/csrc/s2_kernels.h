@@ -53,6 +53,11 @@ constexpr int kGapBuckets = 32;
 int launch_graph_gap(const Plan& p, const float* lse_s, const float* lse_f, const void* o_s, const void* o_f,
                      float* rho, float* dist, float* stats, cudaStream_t stream);
 
+// Halo movement of sequence-parallel ranks (part 0: K/V, 1: gradients; pack:
+// tensors -> message, else message -> tensors, accumulated for gradients).
+int launch_halo(void* a, void* b, void* msg, int B, int L, int H, int D, int G, int part, bool pack,
+                cudaStream_t stream);
+
 // Rotary position prologue on original positions (positions: int32 [B, N] or null = 0..N-1).
 int launch_rope(const void* q, const void* k, void* q_out, void* k_out, const int* positions, int B, int N, int H,
                 int D, double base, double scale, cudaStream_t stream);

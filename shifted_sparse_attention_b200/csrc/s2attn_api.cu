@@ -150,15 +150,15 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 104; }
+int s2attn_version(void) { return 105; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
-static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* docs,
-                    int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
-                    void* stream) {
-  int rc = validate(B, N, H, D, G, n_valid, variant);
-  if (rc) return rc;
+// Pointer checks, tensor maps over [B, plan.N, H, D] and the forward launch.
+static int fwd_launch(const void* q, const void* k, const void* v, void* o, float* lse, const s2::Plan& plan,
+                      void* stream) {
+  int rc;
+  const int64_t B = plan.B, N = plan.N, H = plan.H, D = plan.D;
   if (!q || !k || !v || !o || !lse) return fail(S2_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return fail(S2_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
@@ -170,12 +170,21 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     return rc;
   s2::FwdArgs a;
   a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmO = &to;
-  a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
-  a.plan.docs = docs;
+  a.plan = plan;
   a.lse = lse;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_fwd(a), "forward");
+}
+
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, const int32_t* docs,
+                    int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                    void* stream) {
+  int rc = validate(B, N, H, D, G, n_valid, variant);
+  if (rc) return rc;
+  s2::Plan plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  plan.docs = docs;
+  return fwd_launch(q, k, v, o, lse, plan, stream);
 }
 
 int s2attn_fwd_v(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t N,
@@ -258,13 +267,13 @@ size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
   return 2 * stat_bytes(B, N, H);
 }
 
-static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                    const float* lse, const int32_t* docs, void* dq, void* dk, void* dv, int64_t B, int64_t N,
-                    int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace,
-                    size_t workspace_bytes, int stages, void* stream) {
+// Pointer and workspace checks, tensor maps over [B, plan.N, H, D] and the backward stages.
+static int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, const s2::Plan& plan, void* workspace,
+                      size_t workspace_bytes, int stages, void* stream) {
   if (stages < 1 || stages > S2_BWD_ALL) return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7");
-  int rc = validate(B, N, H, D, G, n_valid, variant);
-  if (rc) return rc;
+  int rc;
+  const int64_t B = plan.B, N = plan.N, H = plan.H, D = plan.D;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
     return fail(S2_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
@@ -285,8 +294,7 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
     return rc;
   s2::BwdArgs a;
   a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmdO = &tdo; a.tmdK = &tdk; a.tmdV = &tdv; a.tmdQ = &tdq;
-  a.plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
-  a.plan.docs = docs;
+  a.plan = plan;
   a.o = o;
   a.dout = dout;
   a.lse = lse;
@@ -296,6 +304,94 @@ static int bwd_impl(const void* q, const void* k, const void* v, const void* o, 
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");
+}
+
+static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, const int32_t* docs, void* dq, void* dk, void* dv, int64_t B, int64_t N,
+                    int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace,
+                    size_t workspace_bytes, int stages, void* stream) {
+  if (stages < 1 || stages > S2_BWD_ALL) return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7");
+  int rc = validate(B, N, H, D, G, n_valid, variant);
+  if (rc) return rc;
+  s2::Plan plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);
+  plan.docs = docs;
+  return bwd_launch(q, k, v, o, dout, lse, dq, dk, dv, plan, workspace, workspace_bytes, stages, stream);
+}
+
+// ------------------------------------------------------------ sequence parallelism
+
+// Shape rules of one rank's call: the method's rules on the shard (L a
+// multiple of G), padding only on the last rank, ROLLED without padding.
+static int validate_sp(int64_t B, int64_t L, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                       int rank, int world) {
+  if (variant != S2_STRICT && variant != S2_ROLLED)
+    return fail(variant == S2_DENSE_CAUSAL ? S2_ERR_UNSUPPORTED : S2_ERR_INVALID_ARG,
+                "sequence parallelism supports the STRICT and ROLLED variants (got %d)", variant);
+  if (world < 1 || rank < 0 || rank >= world)
+    return fail(S2_ERR_INVALID_ARG, "rank %d out of range for world %d", rank, world);
+  int rc = validate(B, L, H, D, G, n_valid, variant);
+  if (rc) return rc;
+  if (n_valid < L && rank != world - 1)
+    return fail(S2_ERR_SHAPE, "only the last rank may hold padding (rank %d of %d, n_valid %lld < L %lld)", rank,
+                world, (long long)n_valid, (long long)L);
+  if (variant == S2_ROLLED && n_valid < L)
+    return fail(S2_ERR_UNSUPPORTED, "ROLLED across ranks needs an unpadded sequence");
+  if (B * (L + G / 2) >= (int64_t(1) << 31) || B * H * (L + G / 2) >= (int64_t(1) << 31))
+    return fail(S2_ERR_UNSUPPORTED, "B*(L+G/2) and B*H*(L+G/2) must be below 2^31");
+  return S2_OK;
+}
+
+static s2::Plan plan_sp(int64_t B, int64_t L, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
+                        int rank) {
+  return s2::make_plan_sp((int)B, (int)L, (int)H, (int)D, (int)G, (int)(G / 2 + n_valid),
+                          variant == S2_STRICT && rank == 0);
+}
+
+int s2attn_sp_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t L,
+                  int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, int rank, int world, void* stream) {
+  int rc = validate_sp(B, L, H, D, G, n_valid, variant, rank, world);
+  if (rc) return rc;
+  return fwd_launch(q, k, v, o, lse, plan_sp(B, L, H, D, G, n_valid, variant, rank), stream);
+}
+
+int s2attn_sp_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+                  void* dq, void* dk, void* dv, int64_t B, int64_t L, int64_t H, int64_t D, int64_t G,
+                  int64_t n_valid, int variant, int rank, int world, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int rc = validate_sp(B, L, H, D, G, n_valid, variant, rank, world);
+  if (rc) return rc;
+  return bwd_launch(q, k, v, o, dout, lse, dq, dk, dv, plan_sp(B, L, H, D, G, n_valid, variant, rank), workspace,
+                    workspace_bytes, S2_BWD_ALL, stream);
+}
+
+size_t s2attn_sp_halo_bytes(int64_t B, int64_t H, int64_t D, int64_t G) {
+  if (B < 1 || H < 2 || D < 1 || G < 2) return 0;
+  return (size_t)(2 * B * (G / 2) * (H / 2) * D * 2);
+}
+
+static int halo_impl(void* a, void* b, void* msg, int64_t B, int64_t L, int64_t H, int64_t D, int64_t G, int part,
+                     bool pack, void* stream) {
+  if (part != S2_SP_KV && part != S2_SP_GRAD) return fail(S2_ERR_INVALID_ARG, "part must be S2_SP_KV or S2_SP_GRAD");
+  int rc = validate(B, L, H, D, G, L, S2_STRICT);
+  if (rc) return rc;
+  if (!a || !b || !msg) return fail(S2_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(a) || !aligned16(b) || !aligned16(msg))
+    return fail(S2_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st))) return rc;
+  return launch_status(s2::launch_halo(a, b, msg, (int)B, (int)L, (int)H, (int)D, (int)G, part, pack,
+                                       static_cast<cudaStream_t>(stream)),
+                       "halo");
+}
+
+int s2attn_sp_halo_pack(const void* a, const void* b, void* msg, int64_t B, int64_t L, int64_t H, int64_t D,
+                        int64_t G, int part, void* stream) {
+  return halo_impl(const_cast<void*>(a), const_cast<void*>(b), msg, B, L, H, D, G, part, true, stream);
+}
+
+int s2attn_sp_halo_unpack(const void* msg, void* a, void* b, int64_t B, int64_t L, int64_t H, int64_t D, int64_t G,
+                          int part, void* stream) {
+  return halo_impl(a, b, const_cast<void*>(msg), B, L, H, D, G, part, false, stream);
 }
 
 int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o, const void* dout,

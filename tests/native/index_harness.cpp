@@ -136,6 +136,74 @@ int s2h_visit_docs(int N, int G, int n_valid, int variant, int cls, const int32_
   return units;
 }
 
+// Sequence-parallel traversal: the pairs computed by rank `rank` of `world`
+// (shards of L rows, plan over the extended buffer of s + L rows whose first
+// s rows are the halo), mapped to GLOBAL positions of the N = world·L
+// sequence: extended row e is global rank·L - s + e (modulo N for ROLLED).
+// visited[gi*N + gj] += 1 per computed pair; `which`: 0 forward, 1 dK/dV,
+// 2 dQ (each walk mirrors its kernel's traversal).  Returns -1 if a pair
+// touches a halo row with no global position (rank 0 of STRICT).
+int s2h_visit_sp(int L, int G, int n_valid_local, int variant, int rank, int world, int cls, int which,
+                 uint8_t* visited) {
+  const int s = G / 2, N = world * L;
+  s2::Plan p = s2::make_plan_sp(1, L, 2, 128, G, s + n_valid_local, variant == s2::kStrict && rank == 0);
+  int bad = 0;
+  auto mark = [&](int qe, int ke) {
+    long long gq = (long long)rank * L - s + qe, gk = (long long)rank * L - s + ke;
+    if (variant == s2::kRolled) { gq = (gq + N) % N; gk = (gk + N) % N; }
+    if (gq < 0 || gk < 0 || gq >= N || gk >= N) { bad = 1; return; }
+    visited[gq * N + gk] += 1;
+  };
+  if (which == 0) {
+    for (int Li = 0; Li < s2::grid_fwd(p); ++Li) {
+      s2::Unit u;
+      if (!s2::decode_unit(p, Li, u) || u.h != cls) continue;
+      for (int x = 0; x < 2; ++x) {
+        if (!u.part[x]) continue;
+        const int q0 = s2::tile_orig(p, u, u.t[x]);
+        for (int k = 0; k <= u.t[x]; ++k) {
+          if (!s2::ktile_valid(p, u, k)) continue;
+          const int k0 = s2::tile_orig(p, u, k);
+          for (int r = 0; r < s2::kTile; ++r) {
+            const int lim = s2::col_limit(p, u, u.t[x], k, r);
+            for (int c = 0; c < lim; ++c) mark(q0 + r, k0 + c);
+          }
+        }
+      }
+    }
+  } else if (which == 1) {
+    for (int Li = 0; Li < s2::grid_bwd(p); ++Li) {
+      s2::Unit u;
+      if (!s2::decode_kv_unit(p, Li, u) || u.h != cls || !u.part[0]) continue;
+      const int kt = u.t[0], k0 = s2::tile_orig(p, u, kt);
+      for (int qt = kt; qt <= u.kmax; ++qt) {  // the kernel starts at the first valid query tile
+        if (!s2::qtile_valid(p, u, qt)) continue;
+        const int q0 = s2::tile_orig(p, u, qt);
+        for (int j = 0; j < s2::kTile; ++j) {
+          int lo, hi;
+          s2::query_range(p, u, kt, qt, j, lo, hi);
+          for (int i = lo; i < hi; ++i) mark(q0 + i, k0 + j);
+        }
+      }
+    }
+  } else {
+    for (int Li = 0; Li < s2::grid_bwd(p); ++Li) {
+      s2::Unit u;
+      if (!s2::decode_q_unit(p, Li, u) || u.h != cls || !u.part[0]) continue;
+      const int qt = u.t[0], q0 = s2::tile_orig(p, u, qt);
+      for (int k = 0; k <= qt; ++k) {
+        if (!s2::ktile_valid(p, u, k)) continue;
+        const int k0 = s2::tile_orig(p, u, k);
+        for (int r = 0; r < s2::kTile; ++r) {
+          const int lim = s2::col_limit(p, u, qt, k, r);
+          for (int c = 0; c < lim; ++c) mark(q0 + r, k0 + c);
+        }
+      }
+    }
+  }
+  return bad ? -1 : 0;
+}
+
 // Grid size and per-class unit counts of a launch.
 void s2h_plan(int B, int N, int H, int G, int n_valid, int variant, int32_t* out) {
   s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);

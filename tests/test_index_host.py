@@ -35,6 +35,8 @@ def harness(tmp_path_factory):
     L.s2h_plan.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p]
     L.s2h_visit_docs.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
     L.s2h_visit_docs.restype = ctypes.c_int
+    L.s2h_visit_sp.argtypes = [ctypes.c_int] * 8 + [ctypes.c_void_p]
+    L.s2h_visit_sp.restype = ctypes.c_int
     return L
 
 
@@ -169,7 +171,7 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 104
+    assert L.s2attn_version() == 105
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
@@ -228,3 +230,61 @@ def test_rope_host_validation(abi):
     assert rc == abi.S2_ERR_INVALID_ARG  # misaligned positions
     rc = L.s2attn_rope(fake, fake, fake, fake, None, 0, 16, 2, 128, 10000.0, 1.0, None)
     assert rc == abi.S2_ERR_SHAPE
+
+
+# ---------------------------------------------------------------- sequence parallelism
+# "4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1: with G-aligned shards and a
+# half-group halo exchange, the multi-rank graph must equal the single-GPU one
+# (the pages' single- vs multi-card comparison of visible sets): the union over
+# ranks of the pairs each rank's kernels compute is exactly A^(0) / A^(1) of
+# the whole sequence, every pair once, in the forward and in both backward passes.
+
+SP_CASES = [(G, L // G, W) for G in (256, 512) for L in (G, 2 * G) for W in (1, 2, 3, 4)]
+
+
+@pytest.mark.parametrize("G,per,W", SP_CASES)
+@pytest.mark.parametrize("variant", [0, 1])
+def test_sequence_parallel_union_is_the_single_gpu_graph(harness, G, per, W, variant):
+    L = G * per
+    N = W * L
+    for nv_last in ([L] if variant == 1 else [L, L - 100, 1]):
+        nv = (W - 1) * L + nv_last
+        for cls in (0, 1):
+            ref = oracle.adjacency(N, G, nv, variant, cls)
+            for which in (0, 1, 2):
+                vis = np.zeros((N, N), dtype=np.uint8)
+                for r in range(W):
+                    rc = harness.s2h_visit_sp(L, G, nv_last if r == W - 1 else L, variant, r, W, cls, which,
+                                              vis.ctypes.data)
+                    assert rc == 0, ("halo row without a global position", r)
+                assert vis.max() <= 1, ("pair computed twice", which)
+                np.testing.assert_array_equal(vis.astype(bool), ref, err_msg=str((W, L, cls, which, nv)))
+
+
+def test_sequence_parallel_host_validation(abi):
+    L = abi.lib()
+    fake = 1 << 20
+    base = dict(B=1, L=1024, H=8, D=128, G=256, nv=1024, variant=0, rank=0, world=2)
+    cases = [
+        (dict(variant=2), abi.S2_ERR_UNSUPPORTED),       # dense causal does not shard by halos
+        (dict(variant=5), abi.S2_ERR_INVALID_ARG),
+        (dict(rank=2), abi.S2_ERR_INVALID_ARG),
+        (dict(world=0), abi.S2_ERR_INVALID_ARG),
+        (dict(L=1000), abi.S2_ERR_SHAPE),                # shard not a multiple of G
+        (dict(nv=1000), abi.S2_ERR_SHAPE),               # padding on a rank that is not the last
+        (dict(nv=1000, rank=1, variant=1), abi.S2_ERR_UNSUPPORTED),  # ROLLED needs no padding
+    ]
+    for over, code in cases:
+        a = dict(base)
+        a.update(over)
+        rc = L.s2attn_sp_fwd(fake, fake, fake, fake, fake, a["B"], a["L"], a["H"], a["D"], a["G"], a["nv"],
+                             a["variant"], a["rank"], a["world"], None)
+        assert rc == code, (over, rc, abi.s2attn_last_error())
+        rc = L.s2attn_sp_bwd(*([fake] * 9), a["B"], a["L"], a["H"], a["D"], a["G"], a["nv"], a["variant"], a["rank"],
+                             a["world"], fake, 1 << 30, None)
+        assert rc == code, (over, rc, abi.s2attn_last_error())
+    assert L.s2attn_sp_halo_bytes(2, 32, 128, 8192) == 2 * 2 * 16 * 4096 * 128 * 2  # V_KV, K and V
+    rc = L.s2attn_sp_halo_pack(fake, fake, fake, 1, 1024, 8, 128, 256, 7, None)
+    assert rc == abi.S2_ERR_INVALID_ARG
+    rc = L.s2attn_sp_halo_unpack(fake, fake, fake + 8, 1, 1024, 8, 128, 256, 0, None)
+    assert rc == abi.S2_ERR_INVALID_ARG
