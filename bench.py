@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--doc-len", type=int, default=0,
                     help="pack documents of this many tokens (document mask); reports exact-pair TFLOP/s")
+    ap.add_argument("--sp-emulate", type=int, default=0, metavar="W",
+                    help="sequence parallelism: run W ranks' shards (halo exchange + rank kernels) in turn on this GPU")
     ap.add_argument("--rope", action="store_true",
                     help="start each step with the RoPE prologue (original positions, interpolation 1/4)")
     return ap.parse_args()
@@ -479,6 +481,115 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_sp_emulated(args):
+    """Sequence-parallel step of W ranks, run one rank after another on this GPU.
+
+    Each rank holds a G-aligned shard of L = N / W rows of the workload in
+    extended buffers; per step and rank: K/V halo from the previous rank
+    (pack + unpack kernels, the message handed over in memory where the
+    collective layer would send it), the rank's forward and backward, and the
+    halo gradients back (pack + accumulate).  value = the whole sequence's
+    useful FLOPs / the summed device time of all ranks (comparable with the
+    single-GPU line); per_rank_ms is what each GPU of a W-GPU job would spend
+    on kernels, without the transfer itself (estimated from the halo bytes at
+    the measured 770 GB/s peer bandwidth)."""
+    import torch
+
+    from shifted_sparse_attention_b200 import binding as s2
+    from shifted_sparse_attention_b200 import sp
+    from shifted_sparse_attention_b200 import synthetic
+
+    torch.cuda.set_device(0)
+    w = synthetic.WORKLOADS[args.workload]
+    variant = w.variants[0] if args.variant is None else args.variant
+    B, N, H, D, G, W = w.B, w.N, w.H, w.D, w.G, args.sp_emulate
+    if N % (W * G) or w.valid != N or variant not in (0, 1):
+        raise SystemExit("--sp-emulate needs N divisible by W·G, no padding, strict or rolled")
+    L, s = N // W, G // 2
+    x = synthetic.draw(B, N, H, D, seed=w.seed, sharpen_k=w.sharpen_k)
+    ops = sp.HaloOps()
+    ranks = []
+    for r in range(W):
+        t = {}
+        for name in ("q", "k", "v", "dout"):
+            e = sp.extended(B, L, H, D, G, "cuda")
+            e.zero_()
+            sp.shard(e, G).copy_(x[name][:, r * L:(r + 1) * L])
+            t[name] = e
+        t["o"] = torch.empty_like(t["q"])
+        t["lse"] = torch.empty((B, H, s + L), dtype=torch.float32, device="cuda")
+        t["g"] = tuple(torch.empty_like(t["q"]) for _ in range(3))
+        t["ws"] = torch.empty(s2.s2attn_bwd_workspace_size(B, s + L, H, D), dtype=torch.uint8, device="cuda")
+        ranks.append(t)
+    del x
+    msg = torch.empty((2, B, s, H // 2, D), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def rank_step(r, ev=None):
+        t = ranks[r]
+        to, frm = sp.peers(r, W, variant)
+        if ev is not None:
+            ev[0].record(stream)
+        if frm is not None:
+            f = ranks[frm]
+            ops.pack(f["k"], f["v"], msg, B, L, H, D, G, s2.S2_SP_KV)
+            ops.unpack(msg, t["k"], t["v"], B, L, H, D, G, s2.S2_SP_KV)
+        if ev is not None:
+            ev[1].record(stream)
+        s2._check(s2.s2attn_sp_fwd(t["q"], t["k"], t["v"], t["o"], t["lse"], B, L, H, D, G, L, variant, r, W))
+        dq, dk, dv = t["g"]
+        s2._check(s2.s2attn_sp_bwd(t["q"], t["k"], t["v"], t["o"], t["dout"], t["lse"], dq, dk, dv, B, L, H, D, G,
+                                   L, variant, r, W, t["ws"], t["ws"].numel()))
+        if ev is not None:
+            ev[2].record(stream)
+        if frm is not None:
+            f = ranks[frm]
+            ops.pack(dk, dv, msg, B, L, H, D, G, s2.S2_SP_GRAD)
+            ops.unpack(msg, f["g"][1], f["g"][2], B, L, H, D, G, s2.S2_SP_GRAD)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        for r in range(W):
+            rank_step(r)
+    torch.cuda.synchronize()
+    s2.check_status()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(W)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0") as clk:
+        time.sleep(0.6)
+        start.record(stream)
+        for i in range(args.steps):
+            for r in range(W):
+                rank_step(r, evs[i][r])
+        end.record(stream)
+        torch.cuda.synchronize()
+    s2.check_status()
+    ms_step = start.elapsed_time(end) / args.steps
+    per_rank = [sum(e[r][0].elapsed_time(e[r][3]) for e in evs) / args.steps for r in range(W)]
+    halo = [sum(e[r][0].elapsed_time(e[r][1]) + e[r][2].elapsed_time(e[r][3]) for e in evs) / args.steps
+            for r in range(W)]
+    flops = w.formula_flops(passes="fwd+bwd")
+    pk = peaks()
+    v_kv = s2.s2attn_sp_halo_bytes(B, H, D, G)
+    value = flops / (ms_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC + " (sequence parallel, ranks emulated in turn on one GPU)",
+        "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(_config(w, variant), parallelism="sp%d-emulated" % W, shard_rows=L),
+        "pct_of_peak": {"bf16_burst": value / pk["bf16_burst"], "bf16_sustained": value / pk["bf16_sustained"]},
+        "sp": {"world": W, "per_rank_ms": per_rank, "halo_kernels_ms": halo,
+               "halo_bytes_per_direction": v_kv,
+               "halo_transfer_us_at_770GBps": v_kv / 770e9 * 1e6,
+               "ideal_w_gpu_step_ms": max(per_rank) + 2 * v_kv / 770e9 * 1e3},
+        "clocks": clk.summary(),
+        "gpu_launches": args.steps * sum((6 if sp.peers(r, W, variant)[1] is not None else 2) + 2 for r in range(W)),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -488,6 +599,11 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.sp_emulate:
+        if world > 1:
+            raise SystemExit("--sp-emulate runs on one GPU")
+        run_sp_emulated(args)
         return
     if world > 1:
         import datetime
