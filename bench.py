@@ -49,6 +49,8 @@ def parse():
                     help="pack documents of this many tokens (document mask); reports exact-pair TFLOP/s")
     ap.add_argument("--sp-emulate", type=int, default=0, metavar="W",
                     help="sequence parallelism: run W ranks' shards (halo exchange + rank kernels) in turn on this GPU")
+    ap.add_argument("--recompute-dq", action="store_true",
+                    help="dQ pass recomputes S and dP (8 MB workspace) instead of reading the stored dS")
     ap.add_argument("--rope", action="store_true",
                     help="start each step with the RoPE prologue (original positions, interpolation 1/4)")
     return ap.parse_args()
@@ -79,6 +81,28 @@ def doc_pair_counts(w, variant, doc_len):
         return pairs({0, N}), pairs({0, N})
     s = G // 2
     return pairs(set(range(0, N + 1, G))), pairs({0, N} | set(range(s, N, G)))
+
+
+def stored_tile_pairs(w, variant, cls):
+    """128x128 tile pairs (key tile <= query tile, both holding a valid row) of one
+    head of class cls: the dS tiles the stored-dS backward writes and reads."""
+    N, G, nv, T = w.N, w.G, w.valid, 128
+    if variant == 2:
+        segs = [(0, N)]
+    elif cls == 1 and variant == 0:
+        s = G // 2
+        segs = [(0, s)] + [(s + k * G, G) for k in range(N // G - 1)] + [(N - s, s)]
+    else:
+        segs = [(k * G, G) for k in range(N // G)]  # rolled class 1: padding sits in the wrap group
+    total = 0
+    for start, length in segs:
+        first = [(start + r * T + (G // 2 if variant == 1 and cls == 1 else 0)) % N for r in range(length // T)]
+        valid = [x < nv for x in first]
+        seen = 0
+        for v in valid:  # pairs key tile <= query tile, both valid
+            seen += v
+            total += seen if v else 0
+    return total
 
 
 def pair_counts(w, variant):
@@ -302,7 +326,10 @@ def run_ours(args, rank, world, local_rank):
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     grads = (torch.empty_like(q), torch.empty_like(q), torch.empty_like(q))
-    ws = torch.empty(s2.s2attn_bwd_workspace_size(B, N, H, D), dtype=torch.uint8, device=dev)
+    stored = not args.recompute_dq
+    ws_bytes = (s2.s2attn_bwd_ds_workspace_size(B, N, H, D, G, variant) if stored
+                else s2.s2attn_bwd_workspace_size(B, N, H, D))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     nv = w.n_valid
     docs = None
@@ -331,15 +358,15 @@ def run_ours(args, rank, world, local_rank):
         if ev is not None:
             ev[1].record(stream)
         s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE,
-                    docs=docs)
+                    docs=docs, stored_ds=stored)
         if ev is not None:
             ev[2].record(stream)
         s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DKDV,
-                    docs=docs)
+                    docs=docs, stored_ds=stored)
         if ev is not None:
             ev[3].record(stream)
         s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ,
-                    docs=docs)
+                    docs=docs, stored_ds=stored)
         if ev is not None:
             ev[4].record(stream)
 
@@ -443,7 +470,8 @@ def run_ours(args, rank, world, local_rank):
     algo = pairs * per_pair if pairs is not None else share * w.formula_flops(passes="fwd" if dom == "fwd" else "bwd")
     achieved = algo / (per[dom] * 1e-3) / 1e12
     src = {"fwd": "s2_fwd.cu", "bwd_dkdv": "s2_bwd.cu", "bwd_dq": "s2_bwd.cu"}[dom]
-    kname = {"fwd": "s2_fwd_kernel", "bwd_dkdv": "s2_bwd_dkdv_kernel", "bwd_dq": "s2_bwd_dq_kernel"}[dom]
+    kname = {"fwd": "s2_fwd_kernel", "bwd_dkdv": "s2_bwd_dkdv_kernel",
+             "bwd_dq": "s2_bwd_dq_ds_kernel" if stored else "s2_bwd_dq_kernel"}[dom]
     roof = {"bound": "tensor", "kernel": kname,
             "achieved": achieved, "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
             "frac": achieved / pk["bf16_sustained"],
@@ -469,6 +497,19 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
     }
+    line["config"]["backward"] = ("stored dS (dQ pass reads the dK/dV pass's dS tiles; workspace %.2f GB)"
+                                  % (ws_bytes / 1e9) if stored else "recomputing dQ pass (workspace %.1f MB)"
+                                  % (ws_bytes / 1e6))
+    if stored and not args.doc_len:
+        # the stored-dS dQ pass is HBM-bound: it reads one 32 KB dS tile per computed
+        # tile pair, the K tiles and writes dq
+        tiles = w.B * (w.H // 2) * (stored_tile_pairs(w, variant, 0) + stored_tile_pairs(w, variant, 1))
+        dq_bytes = tiles * 128 * 128 * 2 + 2 * q.numel() * q.element_size()
+        ach = dq_bytes / (per["bwd_dq"] * 1e-3) / 1e9
+        line["dq_roofline"] = {"bound": "hbm", "kernel": "s2_bwd_dq_ds_kernel", "achieved": ach, "peak": pk["hbm_gbs"],
+                               "unit": "GB/s", "frac": ach / pk["hbm_gbs"], "algorithmic_bytes_per_launch": dq_bytes,
+                               "stored_ds_tiles": tiles, "avg_launch_ms": per["bwd_dq"],
+                               "traffic": _traffic("s2_bwd_dq_ds_kernel", "s2_bwd.cu")}
     if args.rope:
         # HBM-bound prologue: reads and writes Q and K once (plus the positions)
         rope_bytes = 2 * 2 * q.numel() * q.element_size() + (positions.numel() * 4 if positions is not None else 0)

@@ -112,6 +112,22 @@ int s2attn_bwd_v(const void* q, const void* k, const void* v, const void* o, con
  * atomic accumulation. */
 enum { S2_BWD_PREPARE = 1, S2_BWD_DKDV = 2, S2_BWD_DQ = 4, S2_BWD_ALL = 7 };
 
+/* Stored-dS backward: adding S2_BWD_STORE_DS to `stages` makes the dK/dV
+ * stage also write every computed 128x128 tile of dS = P∘(dP − Delta) (bf16)
+ * into the workspace, and the dQ stage compute dq = (1/√D)·dS·K from those
+ * tiles instead of recomputing S and dP (both stages of one call sequence
+ * must carry the flag).  The dQ stage then does no exponentials and a third
+ * of the tensor work, and streams the stored tiles from HBM.  The workspace
+ * must then hold s2attn_bwd_ds_workspace_size(B, N, H, D, G, variant) bytes
+ * (the row statistics plus 32 KB per computed tile pair: about N·G·H·B
+ * bytes, 8.7 GB at B1 H32 N32768 G8192).  Results equal the recompute path
+ * within rounding (dS is the same bf16 operand; S and dP come from the dK/dV
+ * pass's products instead of the dQ pass's own), and are bitwise
+ * reproducible run to run. */
+enum { S2_BWD_STORE_DS = 8, S2_BWD_ALL_DS = 15 };
+
+size_t s2attn_bwd_ds_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int variant);
+
 int s2attn_bwd_stages_v(const void* q, const void* k, const void* v, const void* o,
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
                         int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
@@ -276,7 +292,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 105. */
+/* ABI version of this header (major*100 + minor): 106. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

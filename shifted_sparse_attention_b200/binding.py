@@ -23,6 +23,7 @@ SIGNATURES = {
     "s2attn_fwd": ([_vp, _vp, _vp, _vp, _fp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_fwd_v": ([_vp, _vp, _vp, _vp, _fp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_bwd_workspace_size": ([_i64, _i64, _i64, _i64], _sz),
+    "s2attn_bwd_ds_workspace_size": ([_i64, _i64, _i64, _i64, _i64, _int], _sz),
     "s2attn_bwd": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int,
                     _vp, _sz, _vp], _int),
     "s2attn_bwd_v": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64,
@@ -125,6 +126,11 @@ def s2attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, variant, worksp
 
 
 S2_BWD_PREPARE, S2_BWD_DKDV, S2_BWD_DQ, S2_BWD_ALL = 1, 2, 4, 7
+S2_BWD_STORE_DS, S2_BWD_ALL_DS = 8, 15
+
+
+def s2attn_bwd_ds_workspace_size(B, N, H, D, G, variant) -> int:
+    return int(lib().s2attn_bwd_ds_workspace_size(B, N, H, D, G, variant))
 
 
 def s2attn_bwd_stages_v(q, k, v, o, dout, lse, dq, dk, dv, B, N, H, D, G, n_valid, variant, workspace,
@@ -291,14 +297,21 @@ def forward(q, k, v, G: int, variant: int = STRICT, n_valid: int | None = None, 
 
 
 def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int | None = None,
-             grads=None, workspace=None, stream=None, stages: int = 7, docs=None):
-    """S²-Attn backward; returns (dq, dk, dv) bf16 [B,N,H,D].  docs as for forward."""
+             grads=None, workspace=None, stream=None, stages: int = 7, docs=None, stored_ds: bool = False):
+    """S²-Attn backward; returns (dq, dk, dv) bf16 [B,N,H,D].  docs as for forward.
+    stored_ds: the dK/dV stage keeps dS and the dQ stage reads it (adds
+    S2_BWD_STORE_DS to `stages`; the workspace must then be of
+    s2attn_bwd_ds_workspace_size bytes)."""
     B, N, H, D = _shape(q)
     nv = N if n_valid is None else int(n_valid)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dv = grads
-    ws_bytes = s2attn_bwd_workspace_size(B, N, H, D)
+    if stored_ds:
+        stages |= S2_BWD_STORE_DS
+        ws_bytes = s2attn_bwd_ds_workspace_size(B, N, H, D, G, variant)
+    else:
+        ws_bytes = s2attn_bwd_workspace_size(B, N, H, D)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
     wb = workspace.numel() * workspace.element_size()

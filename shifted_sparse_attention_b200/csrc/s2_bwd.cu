@@ -187,13 +187,15 @@ struct Layout {
 
 }  // namespace dkdv
 
-template <int D>
+// kStoreDS: also write every dS tile (bf16, key rows x query columns) to
+// `ds_store` for the stored-dS dQ pass.
+template <int D, bool kStoreDS>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     s2_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                        const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                        const __grid_constant__ Plan p, const float* __restrict__ delta,
-                       const float* __restrict__ lse2,
+                       const float* __restrict__ lse2, __nv_bfloat16* __restrict__ ds_store,
                        int* __restrict__ status) {
   using namespace bwd;
   using namespace dkdv;
@@ -426,6 +428,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       while (ok && qt >= 0) {
         const int sd = n % kOSlots;
         const int qn = next_q(p, u, qt, lK, hK);
+        // stored dS: row j of tile (qt, kt), query columns [64x, 64x + 64)
+        uint4* ds_row = nullptr;
+        if constexpr (kStoreDS)
+          ds_row = reinterpret_cast<uint4*>(ds_store + (ds_slot(p, u, qt, kt) * kTile + j) * kTile + 64 * x);
         // dS(n) = P (dP - Delta) -> dS^T pairs into R2
         ok = s2_wait(bar(O_FULL + sd), (n / kOSlots) & 1, abort_flag, status, 32);
         if (ok) ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
@@ -446,6 +452,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             dsp[i] = pack_bf16(ds.x, ds.y);
           }
           tmem_st16(tR2 + lane_off + 64 * x + 16 * c, dsp);
+          if constexpr (kStoreDS) {
+            // evict-first: the dQ pass reads these tiles after the whole pass
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              __stcs(ds_row + 4 * c + v4, make_uint4(dsp[4 * v4], dsp[4 * v4 + 1], dsp[4 * v4 + 2], dsp[4 * v4 + 3]));
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -803,12 +815,188 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #undef sVs
 }
 
+// ------------------------------------------------------------------ dQ from stored dS
+// One CTA per 128-query tile: dQ = sum over the unit's key tiles of dS K,
+// with dS read back from the dK/dV pass (transposed tiles: key rows, query
+// columns, so dS enters the MMA as an MN-major A operand) and K as an
+// MN-major B operand.  No exponentials, no recomputed products: the pass
+// streams 32 KB of dS per key tile from HBM and is bounded by that.  Warp 8
+// loads (dS tile + K tile per stage, three stages), one thread of warp 9
+// issues the MMAs, warps 0-7 run the epilogue (dq = bf16(dQ/sqrt(D)) through
+// a TMA store).
+namespace dqs {
+
+constexpr int kStages = 3;
+enum Bar { FULL = 0, EMPTY = 3, DQ_DONE = 6, NUM_BARS = 7 };
+
+template <int D>
+struct Layout {
+  static constexpr int kDSBytes = kTile * kTile * 2;
+  static constexpr int kKBytes = kTile * D * 2;
+  static constexpr int kStageBytes = kDSBytes + kKBytes;
+  static constexpr int kBars = kStages * kStageBytes;
+  static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
+};
+
+}  // namespace dqs
+
+template <int D>
+__global__ void __launch_bounds__(bwd::kThreads, 1)
+    s2_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmDS,
+                        const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ Plan p,
+                        int* __restrict__ status) {
+  using namespace bwd;
+  using namespace dqs;
+  using L = dqs::Layout<D>;
+  constexpr int kChunks = D / 64;
+
+  Unit u;
+  if (!decode_q_unit(p, blockIdx.x, u)) return;
+  extern __shared__ __align__(1024) uint8_t smem_dqs[];
+  if (smem_u32(smem_dqs) & 1023u) {
+    if (threadIdx.x == 0) atomicOr(status, 256);
+    return;
+  }
+  const int qt = u.t[0];
+  const int q0 = tile_orig(p, u, qt);
+  const bool qvalid = u.part[0];
+  int lQ = 0, hQ = p.N;
+  if (qvalid) doc_span(p, u.b, q0, lQ, hQ);
+
+  uint8_t* smem = smem_dqs;
+  const uint32_t sb = smem_u32(smem);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t sbar = sb + L::kBars;
+#define bar(i) (sbar + 8u * (uint32_t)(i))
+#define sDS(st) (sb + (uint32_t)(st) * L::kStageBytes)
+#define sKt(st) (sb + (uint32_t)(st) * L::kStageBytes + L::kDSBytes)
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(bar(FULL + i), 1);
+      mbar_init(bar(EMPTY + i), 1);
+    }
+    mbar_init(bar(DQ_DONE), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), D);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tdQ = *tmem_slot;
+  const int row_base = u.b * p.N;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && qvalid) {
+      prefetch_tmap(&tmDS);
+      prefetch_tmap(&tmK);
+      int e = 0;
+      bool ok = true;
+      for (int k = next_k(p, u, -1, lQ, hQ); ok && k >= 0; k = next_k(p, u, k, lQ, hQ), ++e) {
+        const int st = e % kStages;
+        if (e >= kStages) ok = s2_wait(bar(EMPTY + st), ((e / kStages) - 1) & 1, abort_flag, status, 1);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bar(FULL + st), L::kStageBytes);
+        const int ds_row = (int)(ds_slot(p, u, qt, k) * kTile);
+        tma_load_2d(sDS(st), &tmDS, 0, ds_row, bar(FULL + st));
+        tma_load_2d(sDS(st) + kChunkBytes, &tmDS, 64, ds_row, bar(FULL + st));
+        const int row = row_base + tile_orig(p, u, k);
+        for (int c = 0; c < kChunks; ++c) tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
+      }
+      // the last loads must land before the CTA retires
+      for (int d = (e > kStages ? e - kStages : 0); d < e; ++d)
+        s2_wait(bar(FULL + d % kStages), (d / kStages) & 1, abort_flag, status, 1);
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && qvalid) {
+      // dQ: M = 128 queries, N = D, K = 128 keys; A = dS (MN-major: queries contiguous), B = K (MN-major)
+      constexpr uint32_t id_q = umma_idesc_bf16(128, D, 1, 1);
+      const uint64_t dDS_mn = umma_desc_sw128(sDS(0), kChunkBytes, 1024);
+      const uint64_t dK_mn = umma_desc_sw128(sKt(0), kChunkBytes, 1024);
+      constexpr uint64_t kStageStep = (uint64_t)(L::kStageBytes >> 4);
+      bool ok = true;
+      int jj = 0;
+      for (int k = next_k(p, u, -1, lQ, hQ); ok && k >= 0; k = next_k(p, u, k, lQ, hQ), ++jj) {
+        const int st = jj % kStages;
+        ok = s2_wait(bar(FULL + st), (jj / kStages) & 1, abort_flag, status, 2);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t so = (uint64_t)st * kStageStep;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_ss(tdQ, dDS_mn + so + S2_MN_OFF(kk), dK_mn + so + S2_MN_OFF(kk), id_q, (jj > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(EMPTY + st));
+      }
+      // every issued MMA must be complete before TMEM is read or released
+      umma_commit(bar(DQ_DONE));
+      s2_wait(bar(DQ_DONE), 0, abort_flag, status, 2);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue: dq
+    const int x = warp / 4;
+    const int r = (warp % 4) * 32 + lane;
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    const bool row_valid = q0 + r < p.n_valid;
+    bool have = qvalid;
+    if (have) {
+      have = s2_wait(bar(DQ_DONE), 0, abort_flag, status, 4);
+      tc_fence_after();
+    }
+    const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
+    // staging in stage 0's dS area (every load has landed and every MMA has completed)
+    acc_to_smem<D>(tdQ, lane_off, x, r, have, row_valid, scale, sDS(0));
+    fence_proxy_async_smem();
+    named_bar_sync(2, 256);
+    if (threadIdx.x == 0) {
+      for (int c = 0; c < kChunks; ++c) tma_store_3d(&tmdQ, sDS(0) + c * kChunkBytes, c * 64, u.h, row_base + q0);
+      tma_store_commit();
+      tma_store_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tdQ, D);
+  }
+#undef bar
+#undef sDS
+#undef sKt
+}
+
 #undef S2_KM_OFF
 #undef S2_MN_OFF
 
+template <int D, bool kStoreDS>
+int launch_dkdv(const BwdArgs& a, int grid) {
+  constexpr int kBytes = dkdv::Layout<D>::kBytes;
+  cudaError_t e =
+      cudaFuncSetAttribute(s2_bwd_dkdv_kernel<D, kStoreDS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+  if (e != cudaSuccess) return (int)e;
+  s2_bwd_dkdv_kernel<D, kStoreDS><<<grid, bwd::kThreads, kBytes, a.stream>>>(
+      *a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK, *a.tmdV, a.plan, a.delta, a.lse2,
+      static_cast<__nv_bfloat16*>(a.ds), a.status);
+  return (int)cudaGetLastError();
+}
+
 template <int D>
 int launch_bwd_impl(const BwdArgs& a, int stages) {
-  static_assert(dkdv::Layout<D>::kBytes <= 232448 && dqp::Layout<D>::kBytes <= 232448, "shared memory budget");
+  static_assert(dkdv::Layout<D>::kBytes <= 232448 && dqp::Layout<D>::kBytes <= 232448 &&
+                    dqs::Layout<D>::kBytes <= 232448,
+                "shared memory budget");
+  const bool stored = (stages & 8) != 0;
   const Plan& p = a.plan;
   const long long rows = (long long)p.B * p.N * p.H;
   cudaError_t e;
@@ -821,16 +1009,16 @@ int launch_bwd_impl(const BwdArgs& a, int stages) {
     if (e != cudaSuccess) return (int)e;
   }
   const int grid = grid_bwd(p);
-  if (stages & 2) {  // dK, dV
-    constexpr int kBytes = dkdv::Layout<D>::kBytes;
-    e = cudaFuncSetAttribute(s2_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
-    if (e != cudaSuccess) return (int)e;
-    s2_bwd_dkdv_kernel<D><<<grid, bwd::kThreads, kBytes, a.stream>>>(*a.tmQ, *a.tmK, *a.tmV, *a.tmdO, *a.tmdK,
-                                                                    *a.tmdV, p, a.delta, a.lse2, a.status);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return (int)e;
+  if (stages & 2) {  // dK, dV (and the stored dS)
+    const int rc = stored ? launch_dkdv<D, true>(a, grid) : launch_dkdv<D, false>(a, grid);
+    if (rc) return rc;
   }
-  if (stages & 4) {  // dQ
+  if ((stages & 4) && stored) {  // dQ from the stored dS
+    constexpr int kBytes = dqs::Layout<D>::kBytes;
+    e = cudaFuncSetAttribute(s2_bwd_dq_ds_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
+    if (e != cudaSuccess) return (int)e;
+    s2_bwd_dq_ds_kernel<D><<<grid, bwd::kThreads, kBytes, a.stream>>>(*a.tmK, *a.tmDS, *a.tmdQ, p, a.status);
+  } else if (stages & 4) {  // dQ
     constexpr int kBytes = dqp::Layout<D>::kBytes;
     e = cudaFuncSetAttribute(s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
     if (e != cudaSuccess) return (int)e;

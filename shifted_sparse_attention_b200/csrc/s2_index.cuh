@@ -62,6 +62,7 @@ struct Plan {
   int off[2];      // segment lattice offset per class (see above)
   int q_begin;     // rows [0, q_begin) are never queries (a sequence-parallel halo)
   int k_begin;     // rows [0, k_begin) hold no valid key
+  long long ds_head_tiles;  // 128x128 dS tiles per (b, h) in the stored-dS backward
   float scale_log2;  // log2(e) / sqrt(D)
   // Packed sequences: per-position document bounds [B, N, 2] = {first position,
   // one past the last position} of the position's document (original
@@ -129,6 +130,7 @@ S2_HD int virt_of(const Plan& p, int cls, int x) {
 // One CTA work unit: up to two consecutive query tiles of one segment.
 struct Unit {
   int b, h, cls;
+  int seg;         // segment index within the head class
   int vbeg;        // virtual start of the segment
   int ntiles;      // query tiles in the segment
   int t[2];        // local tile indices (t[1] = -1 if absent)
@@ -164,6 +166,7 @@ S2_HD bool decode_unit(const Plan& p, int L, Unit& u) {
   if (r >= S * NU) return false;
   const int unit = NU - 1 - r / S;
   const int seg = r % S;
+  u.seg = seg;
   int len;
   seg_bounds(p, u.cls, seg, u.vbeg, len);
   u.ntiles = len / kTile;
@@ -211,6 +214,7 @@ S2_HD bool decode_kv_unit(const Plan& p, int L, Unit& u) {
   const int S = p.nseg[u.cls], NT = p.ntile[u.cls];
   if (r >= S * NT) return false;
   const int kt = r / S, seg = r % S;
+  u.seg = seg;
   int len;
   seg_bounds(p, u.cls, seg, u.vbeg, len);
   u.ntiles = len / kTile;
@@ -236,6 +240,7 @@ S2_HD bool decode_q_unit(const Plan& p, int L, Unit& u) {
   const int S = p.nseg[u.cls], NT = p.ntile[u.cls];
   if (r >= S * NT) return false;
   const int rank = r / S, seg = r % S;
+  u.seg = seg;
   int len;
   seg_bounds(p, u.cls, seg, u.vbeg, len);
   u.ntiles = len / kTile;
@@ -256,6 +261,26 @@ S2_HD void query_range(const Plan& p, const Unit& u, int kt, int qt, int j, int&
   if (tile_orig(p, u, kt) + j >= p.n_valid) { hi = 0; return; }
   const int qv = p.n_valid - tile_orig(p, u, qt);
   hi = qv < kTile ? qv : kTile;
+}
+
+// ---------------------------------------------------------------- stored dS
+// The stored-dS backward keeps every computed 128x128 tile of dS (bf16) from
+// the dK/dV pass for the dQ pass.  Tile (query tile qt, key tile kt <= qt) of
+// a segment sits at slot tri(qt) + kt of the segment's triangle; segments of
+// a head follow each other, heads follow each other (ds_head_tiles apart).
+// A tile is stored transposed, row = key, column = query, as the dK/dV pass
+// produces it (thread = key row).
+S2_HD long long tri(int n) { return (long long)n * (n + 1) / 2; }
+
+S2_HD long long ds_seg_base(const Plan& p, int cls, int seg) {
+  if (p.variant == kDenseCausal) return 0;
+  const int o = p.off[cls], T = p.G / kTile;
+  if (!o) return (long long)seg * tri(T);
+  return seg == 0 ? 0 : tri(o / kTile) + (long long)(seg - 1) * tri(T);
+}
+
+S2_HD long long ds_slot(const Plan& p, const Unit& u, int qt, int kt) {
+  return ((long long)u.b * p.H + u.h) * p.ds_head_tiles + ds_seg_base(p, u.cls, u.seg) + tri(qt) + kt;
 }
 
 // Grid sizes of the forward and backward launches.
@@ -331,6 +356,17 @@ inline void finish_plan(Plan& p) {
   p.hg_fwd = 2;
   p.hg_bwd = 1;
   p.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)p.D));
+  // stored-dS tiles per head: the larger class's sum over segments of tri(tiles)
+  p.ds_head_tiles = 0;
+  for (int c = 0; c < 2; ++c) {
+    long long t = 0;
+    for (int sgi = 0; sgi < p.nseg[c]; ++sgi) {
+      int vb, len;
+      seg_bounds(p, c, sgi, vb, len);
+      t += tri(len / kTile);
+    }
+    if (t > p.ds_head_tiles) p.ds_head_tiles = t;
+  }
 }
 
 // Host-side plan construction (validated by the caller).

@@ -35,12 +35,15 @@ struct BwdArgs {
   const float* lse;   // [B, H, N]
   float* delta;       // workspace [B, H, N]: -(dout_i·o_i)
   float* lse2;        // workspace [B, H, N]: -lse_i·log2(e), -inf on padded rows
+  void* ds;           // stored-dS workspace (bf16 tiles, see s2_index.cuh), or null
+  const CUtensorMap* tmDS;  // 2-D map over the stored dS rows (128 columns), or null
   int* status;
   cudaStream_t stream;
 };
 
 int launch_fwd(const FwdArgs& a);
-// stages: 1 = prepare (Delta, lse2), 2 = dK/dV pass, 4 = dQ pass.
+// stages: 1 = prepare (Delta, lse2), 2 = dK/dV pass, 4 = dQ pass; with 8 the
+// dK/dV pass also stores dS and the dQ pass reads it instead of recomputing.
 int launch_bwd(const BwdArgs& a, int stages);
 // Sets the calling thread's s2attn_last_error() message; returns `code`.
 int report_error(int code, const char* fmt, ...);

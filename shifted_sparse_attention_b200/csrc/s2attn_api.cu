@@ -150,7 +150,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 105; }
+int s2attn_version(void) { return 106; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -267,11 +267,17 @@ size_t s2attn_bwd_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D) {
   return 2 * stat_bytes(B, N, H);
 }
 
+// Bytes of the stored-dS area: one 128x128 bf16 tile per computed tile pair.
+static size_t ds_bytes(const s2::Plan& p) {
+  return (size_t)p.B * p.H * (size_t)p.ds_head_tiles * s2::kTile * s2::kTile * 2;
+}
+
 // Pointer and workspace checks, tensor maps over [B, plan.N, H, D] and the backward stages.
 static int bwd_launch(const void* q, const void* k, const void* v, const void* o, const void* dout,
                       const float* lse, void* dq, void* dk, void* dv, const s2::Plan& plan, void* workspace,
                       size_t workspace_bytes, int stages, void* stream) {
-  if (stages < 1 || stages > S2_BWD_ALL) return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7");
+  if (stages < 1 || stages > S2_BWD_ALL_DS || stages == S2_BWD_STORE_DS)
+    return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7, optionally with S2_BWD_STORE_DS");
   int rc;
   const int64_t B = plan.B, N = plan.N, H = plan.H, D = plan.D;
   if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace)
@@ -281,9 +287,13 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
     return fail(S2_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(S2_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
-  const size_t need = s2attn_bwd_workspace_size(B, N, H, D);
+  const bool stored = (stages & S2_BWD_STORE_DS) != 0;
+  const size_t stats = s2attn_bwd_workspace_size(B, N, H, D);
+  const size_t need = stats + (stored ? ds_bytes(plan) : 0);
   if (workspace_bytes < need)
     return fail(S2_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
+  if (stored && (long long)B * H * plan.ds_head_tiles * s2::kTile >= (1LL << 31))
+    return fail(S2_ERR_UNSUPPORTED, "stored dS needs B*H*tiles*128 below 2^31 rows");
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
@@ -301,16 +311,39 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   const size_t sb = stat_bytes(B, N, H);
   a.delta = static_cast<float*>(workspace);
   a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
+  a.ds = nullptr;
+  a.tmDS = nullptr;
+  CUtensorMap tds;
+  if (stored) {
+    // [rows, 128] bf16, one 128-row block per tile; box 64 columns x 128 rows, 128-byte swizzle
+    a.ds = static_cast<char*>(workspace) + stats;
+    cuuint64_t dims[2] = {(cuuint64_t)s2::kTile, (cuuint64_t)((long long)B * H * plan.ds_head_tiles * s2::kTile)};
+    cuuint64_t strides[1] = {(cuuint64_t)(s2::kTile * 2)};
+    cuuint32_t box[2] = {64, (cuuint32_t)s2::kTile};
+    cuuint32_t elem[2] = {1, 1};
+    CUresult r = st->encode(&tds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.ds, dims, strides, box, elem,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(S2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    a.tmDS = &tds;
+  }
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");
+}
+
+size_t s2attn_bwd_ds_workspace_size(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int variant) {
+  if (validate(B, N, H, D, G, N, variant) != S2_OK) return 0;
+  const s2::Plan p = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)N, variant);
+  return s2attn_bwd_workspace_size(B, N, H, D) + ds_bytes(p);
 }
 
 static int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
                     const float* lse, const int32_t* docs, void* dq, void* dk, void* dv, int64_t B, int64_t N,
                     int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant, void* workspace,
                     size_t workspace_bytes, int stages, void* stream) {
-  if (stages < 1 || stages > S2_BWD_ALL) return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7");
+  if (stages < 1 || stages > S2_BWD_ALL_DS || stages == S2_BWD_STORE_DS)
+    return fail(S2_ERR_INVALID_ARG, "stages must be a non-empty subset of 7, optionally with S2_BWD_STORE_DS");
   int rc = validate(B, N, H, D, G, n_valid, variant);
   if (rc) return rc;
   s2::Plan plan = s2::make_plan((int)B, (int)N, (int)H, (int)D, (int)G, (int)n_valid, variant);

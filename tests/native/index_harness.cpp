@@ -204,6 +204,44 @@ int s2h_visit_sp(int L, int G, int n_valid_local, int variant, int rank, int wor
   return bad ? -1 : 0;
 }
 
+// Stored-dS tile slots: writes[slot] += 1 for every tile pair the dK/dV pass
+// computes (key tile units, query tiles from the first valid one, under the
+// document spans), reads[slot] += 1 for every tile pair the dQ pass reads.
+// Returns B·H·ds_head_tiles (the slot count of the workspace) or -1 if a slot
+// falls outside it.
+long long s2h_ds_slots(int B, int N, int H, int G, int n_valid, int variant, const int32_t* docs, int32_t* writes,
+                       int32_t* reads) {
+  s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);
+  p.docs = docs;
+  const long long total = (long long)B * H * p.ds_head_tiles;
+  bool bad = false;
+  for (int Li = 0; Li < s2::grid_bwd(p); ++Li) {
+    s2::Unit u;
+    if (!s2::decode_kv_unit(p, Li, u) || !u.part[0]) continue;
+    const int kt = u.t[0];
+    int lo, hi;
+    s2::doc_span(p, u.b, s2::tile_orig(p, u, kt), lo, hi);
+    for (int qt = kt; qt <= u.kmax; ++qt) {
+      if (!s2::qtile_valid(p, u, qt) || !s2::tile_meets(s2::tile_orig(p, u, qt), lo, hi)) continue;
+      const long long sl = s2::ds_slot(p, u, qt, kt);
+      if (sl < 0 || sl >= total) bad = true; else writes[sl] += 1;
+    }
+  }
+  for (int Li = 0; Li < s2::grid_bwd(p); ++Li) {
+    s2::Unit u;
+    if (!s2::decode_q_unit(p, Li, u) || !u.part[0]) continue;
+    const int qt = u.t[0];
+    int lo, hi;
+    s2::doc_span(p, u.b, s2::tile_orig(p, u, qt), lo, hi);
+    for (int k = 0; k <= qt; ++k) {
+      if (!s2::ktile_valid(p, u, k) || !s2::tile_meets(s2::tile_orig(p, u, k), lo, hi)) continue;
+      const long long sl = s2::ds_slot(p, u, qt, k);
+      if (sl < 0 || sl >= total) bad = true; else reads[sl] += 1;
+    }
+  }
+  return bad ? -1 : total;
+}
+
 // Grid size and per-class unit counts of a launch.
 void s2h_plan(int B, int N, int H, int G, int n_valid, int variant, int32_t* out) {
   s2::Plan p = s2::make_plan(B, N, H, 128, G, n_valid, variant);

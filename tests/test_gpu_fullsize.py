@@ -1,7 +1,9 @@
 """Parity at the workloads' full sizes, on sampled outputs (needs a B200).
 
 Each workload runs through the C ABI exactly as bench.py launches it (one
-forward, then the backward's three stages) on the full seeded inputs.  The
+forward, then the backward's three stages, with the stored-dS dQ pass as
+bench.py times it, and again with the recomputing dQ pass) on the full
+seeded inputs.  The
 float64 oracle then recomputes windows of 64 query rows for a few heads of
 each class: at segment starts, at segment ends (where the window also holds
 every query that sees the window's keys, so dK and dV are complete there),
@@ -53,12 +55,21 @@ def _windows(w, variant, cls):
     return [(max(0, a), min(N, b), c) for a, b, c in out if b - a > 0 and a < nv]
 
 
-def _check_workload(name, variant):
+@functools.lru_cache(maxsize=64)
+def _oracle_window(name, variant, r0, r1, bhs):
+    w = synthetic.WORKLOADS[name]
+    x = _inputs(w.B, w.N, w.H, w.D, w.seed, w.sharpen_k)
+    return oracle.attention_window(x["q"], x["k"], x["v"], x["dout"], G=w.G, variant=variant, rows=(r0, r1),
+                                   heads=list(bhs), n_valid=w.n_valid)
+
+
+def _check_workload(name, variant, stored=True):
     w = synthetic.WORKLOADS[name]
     x = _inputs(w.B, w.N, w.H, w.D, w.seed, w.sharpen_k)
     dev = {n: t.cuda() for n, t in x.items()}
     o, lse = s2.forward(dev["q"], dev["k"], dev["v"], w.G, variant, w.n_valid)
-    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, w.G, variant, w.n_valid)
+    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, w.G, variant, w.n_valid,
+                             stored_ds=stored)
     torch.cuda.synchronize()
     s2.check_status()
     del dev
@@ -79,8 +90,7 @@ def _check_workload(name, variant):
     for cls, hs in head_sets.items():
         bhs = [(B - 1 if i % 2 else 0) * H + h for i, h in enumerate(hs)]
         for r0, r1, complete in _windows(w, variant, cls):
-            ref = oracle.attention_window(x["q"], x["k"], x["v"], x["dout"], G=w.G, variant=variant,
-                                          rows=(r0, r1), heads=bhs, n_valid=w.n_valid)
+            ref = _oracle_window(name, variant, r0, r1, tuple(bhs))
             for t, bh in enumerate(bhs):
                 b, h = divmod(bh, H)
                 where = "%s variant %d head %d rows [%d, %d)" % (name, variant, h, r0, r1)
@@ -98,24 +108,32 @@ def _check_workload(name, variant):
                     check_grad("dv", to_np(res["dv"][b, r0:r1, h]), ref["dv"][t], where, gmax["dv"])
 
 
+PATHS = pytest.mark.parametrize("stored", [True, False], ids=["stored_ds", "recompute"])
+
+
+@PATHS
 @pytest.mark.parametrize("variant", [0, 1])
-def test_llama7b_layer_n8192_g2048(variant):
-    _check_workload("llama7b_n8192_g2048", variant)
+def test_llama7b_layer_n8192_g2048(variant, stored):
+    _check_workload("llama7b_n8192_g2048", variant, stored)
 
 
-def test_long_context_n32768_g8192():
-    _check_workload("long_n32768_g8192", 0)
+@PATHS
+def test_long_context_n32768_g8192(stored):
+    _check_workload("long_n32768_g8192", 0, stored)
 
 
+@PATHS
 @pytest.mark.parametrize("name", ["sweep_n12288_g6144", "sweep_n12288_g3072", "sweep_n12288_g2048",
                                   "sweep_n12288_g1536"])
-def test_group_ratio_sweep(name):
-    _check_workload(name, 0)
+def test_group_ratio_sweep(name, stored):
+    _check_workload(name, 0, stored)
 
 
-def test_group_ratio_sweep_full_causal():
-    _check_workload("sweep_n12288_full", 2)
+@PATHS
+def test_group_ratio_sweep_full_causal(stored):
+    _check_workload("sweep_n12288_full", 2, stored)
 
 
-def test_ragged_tail_n100000():
-    _check_workload("ragged_n100000_g8192", 0)
+@PATHS
+def test_ragged_tail_n100000(stored):
+    _check_workload("ragged_n100000_g8192", 0, stored)

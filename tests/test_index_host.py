@@ -37,6 +37,8 @@ def harness(tmp_path_factory):
     L.s2h_visit_docs.restype = ctypes.c_int
     L.s2h_visit_sp.argtypes = [ctypes.c_int] * 8 + [ctypes.c_void_p]
     L.s2h_visit_sp.restype = ctypes.c_int
+    L.s2h_ds_slots.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 3
+    L.s2h_ds_slots.restype = ctypes.c_longlong
     return L
 
 
@@ -171,7 +173,7 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 105
+    assert L.s2attn_version() == 106
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
@@ -288,3 +290,65 @@ def test_sequence_parallel_host_validation(abi):
     assert rc == abi.S2_ERR_INVALID_ARG
     rc = L.s2attn_sp_halo_unpack(fake, fake, fake + 8, 1, 1024, 8, 128, 256, 0, None)
     assert rc == abi.S2_ERR_INVALID_ARG
+
+
+# ---------------------------------------------------------------- stored dS
+# The dK/dV pass writes one dS tile per computed tile pair and the dQ pass
+# reads exactly those tiles: every written slot once, the read set equal to the
+# written set (also under document masks and padding), all inside the workspace.
+
+def _tri(n):
+    return n * (n + 1) // 2
+
+
+def _ds_head_tiles(N, G, variant):
+    if variant == 2:
+        return _tri(N // 128)
+    s = G // 2
+    c0 = (N // G) * _tri(G // 128)
+    c1 = c0 if variant == 1 else 2 * _tri(s // 128) + (N // G - 1) * _tri(G // 128)
+    return max(c0, c1)
+
+
+@pytest.mark.parametrize("N,G", [(1024, 256), (1536, 512), (2048, 1024), (1024, 1024)])
+@pytest.mark.parametrize("variant", [0, 1, 2])
+@pytest.mark.parametrize("docs", [False, True])
+def test_stored_ds_slots_written_once_and_read_back(harness, N, G, variant, docs):
+    B, H = 2, 4
+    for nv in (N, N - 77):
+        d = None
+        if docs:
+            ids = np.zeros((B, N), dtype=np.int32)
+            ids[0, 300:] = 1
+            ids[0, 700:] = 2
+            ids[1, 129:] = 1
+            d = np.zeros((B, N, 2), dtype=np.int32)
+            for b in range(B):
+                st = 0
+                for x in range(1, N + 1):
+                    if x == N or ids[b, x] != ids[b, x - 1]:
+                        d[b, st:x] = (st, x)
+                        st = x
+        total = B * H * _ds_head_tiles(N, G, variant)
+        w = np.zeros(total, dtype=np.int32)
+        r = np.zeros(total, dtype=np.int32)
+        got = harness.s2h_ds_slots(B, N, H, G, nv, variant, d.ctypes.data if d is not None else None,
+                                   w.ctypes.data, r.ctypes.data)
+        assert got == total
+        assert w.max() == 1 and r.max() == 1
+        np.testing.assert_array_equal(w, r)
+
+
+def test_stored_ds_workspace_size(abi):
+    L = abi.lib()
+    for (B, N, H, G, variant) in [(1, 32768, 32, 8192, 0), (2, 12288, 32, 12288, 2), (1, 8192, 32, 2048, 1),
+                                  (1, 106496, 32, 8192, 0)]:
+        got = L.s2attn_bwd_ds_workspace_size(B, N, H, 128, G, variant)
+        assert got == 2 * B * H * N * 4 + B * H * _ds_head_tiles(N, G, variant) * 128 * 128 * 2
+    assert L.s2attn_bwd_ds_workspace_size(1, 1000, 8, 128, 256, 0) == 0  # invalid shape
+    fake = 1 << 20
+    rc = L.s2attn_bwd_stages_v(*([fake] * 9), 1, 1024, 8, 64, 256, 1024, 0, fake, 1 << 30, 8, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # the flag alone runs nothing
+    ws = L.s2attn_bwd_ds_workspace_size(1, 1024, 8, 64, 256, 0)
+    rc = L.s2attn_bwd_stages_v(*([fake] * 9), 1, 1024, 8, 64, 256, 1024, 0, fake, ws - 1, 15, None)
+    assert rc == abi.S2_ERR_INVALID_ARG  # workspace too small for the stored dS
