@@ -428,10 +428,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       while (ok && qt >= 0) {
         const int sd = n % kOSlots;
         const int qn = next_q(p, u, qt, lK, hK);
-        // stored dS: row j of tile (qt, kt), query columns [64x, 64x + 64)
-        uint4* ds_row = nullptr;
+        // stored dS of tile (qt, kt): 16-byte blocks (8 query columns) of key row j at
+        // block-major offsets, so a warp's 32 rows of one block are 512 contiguous bytes
+        uint4* ds_tile = nullptr;
         if constexpr (kStoreDS)
-          ds_row = reinterpret_cast<uint4*>(ds_store + (ds_slot(p, u, qt, kt) * kTile + j) * kTile + 64 * x);
+          ds_tile = reinterpret_cast<uint4*>(ds_store + ds_slot(p, u, qt, kt) * (kTile * kTile)) + j;
         // dS(n) = P (dP - Delta) -> dS^T pairs into R2
         ok = s2_wait(bar(O_FULL + sd), (n / kOSlots) & 1, abort_flag, status, 32);
         if (ok) ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
@@ -456,7 +457,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             // evict-first: the dQ pass reads these tiles after the whole pass
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
-              __stcs(ds_row + 4 * c + v4, make_uint4(dsp[4 * v4], dsp[4 * v4 + 1], dsp[4 * v4 + 2], dsp[4 * v4 + 3]));
+              __stcs(ds_tile + (8 * x + 4 * c + v4) * kTile,
+                     make_uint4(dsp[4 * v4], dsp[4 * v4 + 1], dsp[4 * v4 + 2], dsp[4 * v4 + 3]));
           }
         }
         tmem_wait_st();
@@ -817,9 +819,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
 // ------------------------------------------------------------------ dQ from stored dS
 // One CTA per 128-query tile: dQ = sum over the unit's key tiles of dS K,
-// with dS read back from the dK/dV pass (transposed tiles: key rows, query
-// columns, so dS enters the MMA as an MN-major A operand) and K as an
-// MN-major B operand.  No exponentials, no recomputed products: the pass
+// with dS read back from the dK/dV pass and K as an MN-major B operand.  A
+// stored tile holds dS transposed (key rows, query columns) as 16 blocks of
+// 8 query columns, each block 128 key rows x 16 bytes; a 4-D tensor map
+// (column in block, block, key row, tile) turns 8 blocks into one 128-row x
+// 64-column swizzled chunk, so dS enters the MMA as an MN-major A operand.  No exponentials, no recomputed products: the pass
 // streams 32 KB of dS per key tile from HBM and is bounded by that.  Warp 8
 // loads (dS tile + K tile per stage, three stages), one thread of warp 9
 // issues the MMAs, warps 0-7 run the epilogue (dq = bf16(dQ/sqrt(D)) through
@@ -905,9 +909,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (e >= kStages) ok = s2_wait(bar(EMPTY + st), ((e / kStages) - 1) & 1, abort_flag, status, 1);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(FULL + st), L::kStageBytes);
-        const int ds_row = (int)(ds_slot(p, u, qt, k) * kTile);
-        tma_load_2d(sDS(st), &tmDS, 0, ds_row, bar(FULL + st));
-        tma_load_2d(sDS(st) + kChunkBytes, &tmDS, 64, ds_row, bar(FULL + st));
+        // the tile's blocks 0-7 and 8-15 (query columns 0-63, 64-127) as two
+        // 128-row x 64-column swizzled chunks
+        const int slot = (int)ds_slot(p, u, qt, k);
+        tma_load_4d(sDS(st), &tmDS, 0, 0, 0, slot, bar(FULL + st));
+        tma_load_4d(sDS(st) + kChunkBytes, &tmDS, 0, 8, 0, slot, bar(FULL + st));
         const int row = row_base + tile_orig(p, u, k);
         for (int c = 0; c < kChunks; ++c) tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
       }
