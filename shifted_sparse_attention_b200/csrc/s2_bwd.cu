@@ -821,9 +821,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 // One CTA per 128-query tile: dQ = sum over the unit's key tiles of dS K,
 // with dS read back from the dK/dV pass and K as an MN-major B operand.  A
 // stored tile holds dS transposed (key rows, query columns) as 16 blocks of
-// 8 query columns, each block 128 key rows x 16 bytes; a 4-D tensor map
-// (column in block, block, key row, tile) turns 8 blocks into one 128-row x
-// 64-column swizzled chunk, so dS enters the MMA as an MN-major A operand.  No exponentials, no recomputed products: the pass
+// 8 query columns, each block 128 key rows x 16 bytes (2 KB), which is the
+// unswizzled canonical layout of an MN-major operand: 8-row x 16-byte core
+// matrices, 2048 bytes apart along M (queries), 128 bytes apart along K
+// (keys).  One dense TMA box moves a whole 32 KB tile.  No exponentials, no recomputed products: the pass
 // streams 32 KB of dS per key tile from HBM and is bounded by that.  Warp 8
 // loads (dS tile + K tile per stage, three stages), one thread of warp 9
 // issues the MMAs, warps 0-7 run the epilogue (dq = bf16(dQ/sqrt(D)) through
@@ -909,11 +910,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (e >= kStages) ok = s2_wait(bar(EMPTY + st), ((e / kStages) - 1) & 1, abort_flag, status, 1);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(FULL + st), L::kStageBytes);
-        // the tile's blocks 0-7 and 8-15 (query columns 0-63, 64-127) as two
-        // 128-row x 64-column swizzled chunks
+        // the whole tile: 16 blocks of 128 key rows x 8 query columns
         const int slot = (int)ds_slot(p, u, qt, k);
-        tma_load_4d(sDS(st), &tmDS, 0, 0, 0, slot, bar(FULL + st));
-        tma_load_4d(sDS(st) + kChunkBytes, &tmDS, 0, 8, 0, slot, bar(FULL + st));
+        tma_load_3d(sDS(st), &tmDS, 0, 0, 16 * slot, bar(FULL + st));
         const int row = row_base + tile_orig(p, u, k);
         for (int c = 0; c < kChunks; ++c) tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
       }
@@ -927,7 +926,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (lane == 0 && qvalid) {
       // dQ: M = 128 queries, N = D, K = 128 keys; A = dS (MN-major: queries contiguous), B = K (MN-major)
       constexpr uint32_t id_q = umma_idesc_bf16(128, D, 1, 1);
-      const uint64_t dDS_mn = umma_desc_sw128(sDS(0), kChunkBytes, 1024);
+      const uint64_t dDS_mn = umma_desc_noswz(sDS(0), 2048, 128);
       const uint64_t dK_mn = umma_desc_sw128(sKt(0), kChunkBytes, 1024);
       constexpr uint64_t kStageStep = (uint64_t)(L::kStageBytes >> 4);
       bool ok = true;
@@ -940,7 +939,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         const uint64_t so = (uint64_t)st * kStageStep;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_ss(tdQ, dDS_mn + so + S2_MN_OFF(kk), dK_mn + so + S2_MN_OFF(kk), id_q, (jj > 0 || kk > 0) ? 1u : 0u);
+          // K step kk: 16 keys = two 8-row core matrices of dS (256 bytes), 16 rows of K
+          umma_ss(tdQ, dDS_mn + so + (uint64_t)(kk * 16), dK_mn + so + S2_MN_OFF(kk), id_q,
+                  (jj > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(EMPTY + st));
       }
       // every issued MMA must be complete before TMEM is read or released

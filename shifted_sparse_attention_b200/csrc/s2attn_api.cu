@@ -292,8 +292,8 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   const size_t need = stats + (stored ? ds_bytes(plan) : 0);
   if (workspace_bytes < need)
     return fail(S2_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
-  if (stored && (long long)B * H * plan.ds_head_tiles >= (1LL << 31))
-    return fail(S2_ERR_UNSUPPORTED, "stored dS needs fewer than 2^31 tiles");
+  if (stored && 16LL * B * H * plan.ds_head_tiles >= (1LL << 31))
+    return fail(S2_ERR_UNSUPPORTED, "stored dS needs fewer than 2^27 tiles");
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
@@ -315,16 +315,16 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   a.tmDS = nullptr;
   CUtensorMap tds;
   if (stored) {
-    // a tile = 16 blocks of 8 query columns, each block 128 key rows x 16 bytes:
-    // dims (column in block, block, key row, tile), strides 2048 / 16 / 32768 bytes;
-    // box (8, 8, 128, 1) = 8 blocks -> one 128-row x 64-column chunk, 128-byte swizzle
+    // a tile = 16 blocks of 8 query columns, each block 128 key rows x 16 bytes;
+    // dims (column in block, key row, block over all tiles), strides 16 / 2048 bytes;
+    // box (8, 128, 16) = one whole tile, dense (no swizzle)
     a.ds = static_cast<char*>(workspace) + stats;
-    cuuint64_t dims[4] = {8, 16, (cuuint64_t)s2::kTile, (cuuint64_t)((long long)B * H * plan.ds_head_tiles)};
-    cuuint64_t strides[3] = {(cuuint64_t)(s2::kTile * 16), 16, (cuuint64_t)(s2::kTile * s2::kTile * 2)};
-    cuuint32_t box[4] = {8, 8, (cuuint32_t)s2::kTile, 1};
-    cuuint32_t elem[4] = {1, 1, 1, 1};
-    CUresult r = st->encode(&tds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.ds, dims, strides, box, elem,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    cuuint64_t dims[3] = {8, (cuuint64_t)s2::kTile, (cuuint64_t)(16LL * B * H * plan.ds_head_tiles)};
+    cuuint64_t strides[2] = {16, (cuuint64_t)(s2::kTile * 16)};
+    cuuint32_t box[3] = {8, (cuuint32_t)s2::kTile, 16};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = st->encode(&tds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.ds, dims, strides, box, elem,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(S2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
     a.tmDS = &tds;
