@@ -926,7 +926,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (lane == 0 && qvalid) {
       // dQ: M = 128 queries, N = D, K = 128 keys; A = dS (MN-major: queries contiguous), B = K (MN-major)
       constexpr uint32_t id_q = umma_idesc_bf16(128, D, 1, 1);
-      const uint64_t dDS_mn = umma_desc_noswz(sDS(0), 2048, 128);
+      const uint64_t dDS_mn = umma_desc_noswz(sDS(0), 128, 2048);  // K: 128 B, M: 2048 B
       const uint64_t dK_mn = umma_desc_sw128(sKt(0), kChunkBytes, 1024);
       constexpr uint64_t kStageStep = (uint64_t)(L::kStageBytes >> 4);
       bool ok = true;

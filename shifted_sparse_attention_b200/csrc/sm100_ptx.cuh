@@ -214,8 +214,9 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo
 }
 
 // Shared-memory matrix descriptor, no swizzle (canonical layout of 8-row x
-// 16-byte core matrices, each 128 contiguous bytes): for an MN-major operand
-// lbo = byte distance between core matrices adjacent along M/N, sbo = along K.
+// 16-byte core matrices, each 128 contiguous bytes).  For an MN-major operand
+// in this mode the roles are the reverse of the swizzled modes: lbo = byte
+// distance between core matrices adjacent along K, sbo = along M/N.
 __device__ __forceinline__ uint64_t umma_desc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFF);
