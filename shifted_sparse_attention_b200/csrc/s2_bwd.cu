@@ -428,11 +428,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       while (ok && qt >= 0) {
         const int sd = n % kOSlots;
         const int qn = next_q(p, u, qt, lK, hK);
-        // stored dS of tile (qt, kt): 16-byte blocks (8 query columns) of key row j at
-        // block-major offsets, so a warp's 32 rows of one block are 512 contiguous bytes
+        // stored dS of tile (qt, kt): the 16-byte block of key row j and query columns
+        // [8b, 8b + 8) sits at (j / 8)·2048 + b·128 + (j % 8)·16 bytes, so one block
+        // of a warp's 32 rows is four 128-byte runs
         uint4* ds_tile = nullptr;
         if constexpr (kStoreDS)
-          ds_tile = reinterpret_cast<uint4*>(ds_store + ds_slot(p, u, qt, kt) * (kTile * kTile)) + j;
+          ds_tile = reinterpret_cast<uint4*>(ds_store + ds_slot(p, u, qt, kt) * (kTile * kTile)) + (j >> 3) * 128 +
+                    (j & 7);
         // dS(n) = P (dP - Delta) -> dS^T pairs into R2
         ok = s2_wait(bar(O_FULL + sd), (n / kOSlots) & 1, abort_flag, status, 32);
         if (ok) ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             // evict-first: the dQ pass reads these tiles after the whole pass
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
-              __stcs(ds_tile + (8 * x + 4 * c + v4) * kTile,
+              __stcs(ds_tile + (8 * x + 4 * c + v4) * 8,
                      make_uint4(dsp[4 * v4], dsp[4 * v4 + 1], dsp[4 * v4 + 2], dsp[4 * v4 + 3]));
           }
         }
@@ -820,11 +822,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 // ------------------------------------------------------------------ dQ from stored dS
 // One CTA per 128-query tile: dQ = sum over the unit's key tiles of dS K,
 // with dS read back from the dK/dV pass and K as an MN-major B operand.  A
-// stored tile holds dS transposed (key rows, query columns) as 16 blocks of
-// 8 query columns, each block 128 key rows x 16 bytes (2 KB), which is the
-// unswizzled canonical layout of an MN-major operand: 8-row x 16-byte core
-// matrices, 2048 bytes apart along M (queries), 128 bytes apart along K
-// (keys).  One dense TMA box moves a whole 32 KB tile.  No exponentials, no recomputed products: the pass
+// stored tile (32 KB, contiguous) is already the unswizzled canonical layout
+// of an MN-major operand: core matrices of 8 key rows x 8 query columns (128
+// contiguous bytes), 128 bytes apart along M (queries) and 2048 bytes apart
+// along K (keys), so the 16 core matrices one K group reads are 2 KB of
+// consecutive banks.  One bulk copy moves a tile.  No exponentials, no recomputed products: the pass
 // streams 32 KB of dS per key tile from HBM and is bounded by that.  Warp 8
 // loads (dS tile + K tile per stage, three stages), one thread of warp 9
 // issues the MMAs, warps 0-7 run the epilogue (dq = bf16(dQ/sqrt(D)) through
@@ -847,7 +849,7 @@ struct Layout {
 
 template <int D>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
-    s2_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmDS,
+    s2_bwd_dq_ds_kernel(const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16* __restrict__ ds,
                         const __grid_constant__ CUtensorMap tmdQ, const __grid_constant__ Plan p,
                         int* __restrict__ status) {
   using namespace bwd;
@@ -901,7 +903,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && qvalid) {
-      prefetch_tmap(&tmDS);
       prefetch_tmap(&tmK);
       int e = 0;
       bool ok = true;
@@ -910,9 +911,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (e >= kStages) ok = s2_wait(bar(EMPTY + st), ((e / kStages) - 1) & 1, abort_flag, status, 1);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(FULL + st), L::kStageBytes);
-        // the whole tile: 16 blocks of 128 key rows x 8 query columns
-        const int slot = (int)ds_slot(p, u, qt, k);
-        tma_load_3d(sDS(st), &tmDS, 0, 0, 16 * slot, bar(FULL + st));
+        bulk_load(sDS(st), ds + ds_slot(p, u, qt, k) * (kTile * kTile), L::kDSBytes, bar(FULL + st));
         const int row = row_base + tile_orig(p, u, k);
         for (int c = 0; c < kChunks; ++c) tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
       }
@@ -926,7 +925,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (lane == 0 && qvalid) {
       // dQ: M = 128 queries, N = D, K = 128 keys; A = dS (MN-major: queries contiguous), B = K (MN-major)
       constexpr uint32_t id_q = umma_idesc_bf16(128, D, 1, 1);
-      const uint64_t dDS_mn = umma_desc_noswz(sDS(0), 128, 2048);  // K: 128 B, M: 2048 B
+      const uint64_t dDS_mn = umma_desc_noswz(sDS(0), 2048, 128);  // K: 2048 B, M: 128 B
       const uint64_t dK_mn = umma_desc_sw128(sKt(0), kChunkBytes, 1024);
       constexpr uint64_t kStageStep = (uint64_t)(L::kStageBytes >> 4);
       bool ok = true;
@@ -939,8 +938,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         const uint64_t so = (uint64_t)st * kStageStep;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          // K step kk: 16 keys = two 8-row core matrices of dS (256 bytes), 16 rows of K
-          umma_ss(tdQ, dDS_mn + so + (uint64_t)(kk * 16), dK_mn + so + S2_MN_OFF(kk), id_q,
+          // K step kk: 16 keys = two K groups of dS (4096 bytes), 16 rows of K
+          umma_ss(tdQ, dDS_mn + so + (uint64_t)(kk * 256), dK_mn + so + S2_MN_OFF(kk), id_q,
                   (jj > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(EMPTY + st));
       }
@@ -1024,7 +1023,8 @@ int launch_bwd_impl(const BwdArgs& a, int stages) {
     constexpr int kBytes = dqs::Layout<D>::kBytes;
     e = cudaFuncSetAttribute(s2_bwd_dq_ds_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
     if (e != cudaSuccess) return (int)e;
-    s2_bwd_dq_ds_kernel<D><<<grid, bwd::kThreads, kBytes, a.stream>>>(*a.tmK, *a.tmDS, *a.tmdQ, p, a.status);
+    s2_bwd_dq_ds_kernel<D><<<grid, bwd::kThreads, kBytes, a.stream>>>(
+        *a.tmK, static_cast<const __nv_bfloat16*>(a.ds), *a.tmdQ, p, a.status);
   } else if (stages & 4) {  // dQ
     constexpr int kBytes = dqp::Layout<D>::kBytes;
     e = cudaFuncSetAttribute(s2_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);

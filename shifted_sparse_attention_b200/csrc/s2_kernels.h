@@ -35,8 +35,7 @@ struct BwdArgs {
   const float* lse;   // [B, H, N]
   float* delta;       // workspace [B, H, N]: -(dout_i·o_i)
   float* lse2;        // workspace [B, H, N]: -lse_i·log2(e), -inf on padded rows
-  void* ds;           // stored-dS workspace (bf16 tiles, see s2_index.cuh), or null
-  const CUtensorMap* tmDS;  // 2-D map over the stored dS rows (128 columns), or null
+  void* ds;           // stored-dS workspace (bf16 tiles of 32 KB, see s2_index.cuh), or null
   int* status;
   cudaStream_t stream;
 };

@@ -292,8 +292,7 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   const size_t need = stats + (stored ? ds_bytes(plan) : 0);
   if (workspace_bytes < need)
     return fail(S2_ERR_INVALID_ARG, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, need);
-  if (stored && 16LL * B * H * plan.ds_head_tiles >= (1LL << 31))
-    return fail(S2_ERR_UNSUPPORTED, "stored dS needs fewer than 2^27 tiles");
+
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
@@ -311,24 +310,8 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   const size_t sb = stat_bytes(B, N, H);
   a.delta = static_cast<float*>(workspace);
   a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
-  a.ds = nullptr;
-  a.tmDS = nullptr;
-  CUtensorMap tds;
-  if (stored) {
-    // a tile = 16 blocks of 8 query columns, each block 128 key rows x 16 bytes;
-    // dims (column in block, key row, block over all tiles), strides 16 / 2048 bytes;
-    // box (8, 128, 16) = one whole tile, dense (no swizzle)
-    a.ds = static_cast<char*>(workspace) + stats;
-    cuuint64_t dims[3] = {8, (cuuint64_t)s2::kTile, (cuuint64_t)(16LL * B * H * plan.ds_head_tiles)};
-    cuuint64_t strides[2] = {16, (cuuint64_t)(s2::kTile * 16)};
-    cuuint32_t box[3] = {8, (cuuint32_t)s2::kTile, 16};
-    cuuint32_t elem[3] = {1, 1, 1};
-    CUresult r = st->encode(&tds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.ds, dims, strides, box, elem,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(S2_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
-    a.tmDS = &tds;
-  }
+  // stored dS: bf16 tiles of 32 KB after the row statistics (bulk copies need 16-byte alignment)
+  a.ds = stored ? static_cast<char*>(workspace) + stats : nullptr;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");
