@@ -441,6 +441,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const float2* nd = reinterpret_cast<const float2*>(smem + L::kDelta + sd * L::kRowBytes) + 32 * x;
+        uint32_t keep[kStoreDS ? 32 : 1];  // this row's dS pairs, stored after the hand-off
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
@@ -453,20 +454,21 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                 __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[16 * c + i]);
             const float2 ds = __fmul2_rn(make_float2(pf[32 * c + 2 * i], pf[32 * c + 2 * i + 1]), d2);
             dsp[i] = pack_bf16(ds.x, ds.y);
+            if constexpr (kStoreDS) keep[16 * c + i] = dsp[i];
           }
           tmem_st16(tR2 + lane_off + 64 * x + 16 * c, dsp);
-          if constexpr (kStoreDS) {
-            // evict-first: the dQ pass reads these tiles after the whole pass
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              __stcs(ds_tile + (8 * x + 4 * c + v4) * 8,
-                     make_uint4(dsp[4 * v4], dsp[4 * v4 + 1], dsp[4 * v4 + 2], dsp[4 * v4 + 3]));
-          }
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(DS_READY));
         mbar_arrive(bar(O_EMPTY + sd));  // done with the -Delta rows of dO slot sd
+        if constexpr (kStoreDS) {
+          // after the hand-off, so that draining the stores never holds up dK += dS^T Q;
+          // evict-first: the dQ pass reads these tiles after the whole pass
+#pragma unroll
+          for (int v4 = 0; v4 < 8; ++v4)
+            __stcs(ds_tile + (8 * x + v4) * 8, make_uint4(keep[4 * v4], keep[4 * v4 + 1], keep[4 * v4 + 2], keep[4 * v4 + 3]));
+        }
         if (qn >= 0) {
           ok = p_step(n + 1, qn);
           if (!ok) break;
