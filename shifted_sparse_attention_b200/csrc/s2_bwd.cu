@@ -382,8 +382,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (kvalid) {
       const bool key_tile_ragged = k0 + kTile > p.n_valid;
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
-      float pf[64];  // P of the current tile (fp32), from its exponentials to its dS
-      // P(nn): S^T -> P^T (bf16 pairs into R1) and pf
+      // P of the current tile as bf16 pairs, from its exponentials to its dS: dS uses
+      // the same rounded P as dV += P^T dO
+      uint32_t pk[32];
+      // P(nn): S^T -> P^T (bf16 pairs into R1 and pk); both 32-column loads are in
+      // flight before the one wait
       auto p_step = [&](int nn, int qtile) -> bool {
         const int sq = nn % kQSlots;
         // masks on the diagonal tile, on a key tile with padding and under a
@@ -395,29 +398,25 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!s2_wait(bar(S_FULL), nn & 1, abort_flag, status, 32)) return false;
         tc_fence_after();
         const float2* nl = reinterpret_cast<const float2*>(smem + L::kLse + sq * L::kRowBytes) + 32 * x;
+        uint32_t sv[64];
+        tmem_ld32(tR1 + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tR1 + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {  // 32 query columns at a time
-          uint32_t sv[32];
-          tmem_ld32(tR1 + lane_off + 64 * x + 32 * c, sv);
-          tmem_wait_ld();
-          uint32_t pp[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            // P = 2^(S·log2(e)/sqrt(D) - lse·log2(e)), two columns at a time
-            const float2 a =
-                __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl[16 * c + i]);
-            float p0 = ex2(a.x), p1 = ex2(a.y);
-            if (masked) {
-              const int col = 64 * x + 32 * c + 2 * i;
-              p0 = (col >= lo && col < hi) ? p0 : 0.f;
-              p1 = (col + 1 >= lo && col + 1 < hi) ? p1 : 0.f;
-            }
-            pf[32 * c + 2 * i] = p0;
-            pf[32 * c + 2 * i + 1] = p1;
-            pp[i] = pack_bf16(p0, p1);
+        for (int i = 0; i < 32; ++i) {
+          // P = 2^(S·log2(e)/sqrt(D) - lse·log2(e)), two columns at a time
+          const float2 a = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl[i]);
+          float p0 = ex2(a.x), p1 = ex2(a.y);
+          if (masked) {
+            const int col = 64 * x + 2 * i;
+            p0 = (col >= lo && col < hi) ? p0 : 0.f;
+            p1 = (col + 1 >= lo && col + 1 < hi) ? p1 : 0.f;
           }
-          tmem_st16(tR1 + lane_off + 64 * x + 16 * c, pp);
+          pk[i] = pack_bf16(p0, p1);
         }
+        // P^T pairs over the S columns [64x, 64x + 32), all read already
+        tmem_st16(tR1 + lane_off + 64 * x, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(tR1 + lane_off + 64 * x + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(P_READY));
@@ -441,23 +440,20 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const float2* nd = reinterpret_cast<const float2*>(smem + L::kDelta + sd * L::kRowBytes) + 32 * x;
-        uint32_t keep[kStoreDS ? 32 : 1];  // this row's dS pairs, stored after the hand-off
+        uint32_t dp[64];
+        tmem_ld32(tR2 + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tR2 + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_wait_ld();
+        uint32_t keep[32];  // this row's dS pairs (also stored after the hand-off)
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t dp[32];
-          tmem_ld32(tR2 + lane_off + 64 * x + 32 * c, dp);
-          tmem_wait_ld();
-          uint32_t dsp[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 d2 =
-                __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[16 * c + i]);
-            const float2 ds = __fmul2_rn(make_float2(pf[32 * c + 2 * i], pf[32 * c + 2 * i + 1]), d2);
-            dsp[i] = pack_bf16(ds.x, ds.y);
-            if constexpr (kStoreDS) keep[16 * c + i] = dsp[i];
-          }
-          tmem_st16(tR2 + lane_off + 64 * x + 16 * c, dsp);
+        for (int i = 0; i < 32; ++i) {
+          const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[i]);
+          const float2 pv = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u));
+          const float2 ds = __fmul2_rn(pv, d2);
+          keep[i] = pack_bf16(ds.x, ds.y);
         }
+        tmem_st16(tR2 + lane_off + 64 * x, *reinterpret_cast<const uint32_t(*)[16]>(&keep[0]));
+        tmem_st16(tR2 + lane_off + 64 * x + 16, *reinterpret_cast<const uint32_t(*)[16]>(&keep[16]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(DS_READY));
