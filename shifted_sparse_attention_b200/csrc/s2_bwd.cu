@@ -746,43 +746,42 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         ok = s2_wait(bar(S_FULL + (jj % 2)), (jj / 2) & 1, abort_flag, status, 4);
         if (!ok) break;
         tc_fence_after();
-        float pf[64];
+        // both 32-column loads in flight before one wait; P kept as the bf16 pairs
+        // dS is formed from (the same rounding as the dK/dV pass)
+        uint32_t sv[64];
+        tmem_ld32(tS + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(tS + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_wait_ld();
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t sv[32];
-          tmem_ld32(tS + lane_off + 64 * x + 32 * c, sv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 a = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl2);
-            float p0 = ex2(a.x), p1 = ex2(a.y);
-            if (masked) {
-              const int col = 64 * x + 32 * c + 2 * i;
-              p0 = (col >= cmin && col < cmax) ? p0 : 0.f;
-              p1 = (col + 1 >= cmin && col + 1 < cmax) ? p1 : 0.f;
-            }
-            pf[32 * c + 2 * i] = p0;
-            pf[32 * c + 2 * i + 1] = p1;
+        for (int i = 0; i < 32; ++i) {
+          const float2 a = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl2);
+          float p0 = ex2(a.x), p1 = ex2(a.y);
+          if (masked) {
+            const int col = 64 * x + 2 * i;
+            p0 = (col >= cmin && col < cmax) ? p0 : 0.f;
+            p1 = (col + 1 >= cmin && col + 1 < cmax) ? p1 : 0.f;
           }
+          pk[i] = pack_bf16(p0, p1);
         }
         ok = s2_wait(bar(DP_FULL), jj & 1, abort_flag, status, 4);
         if (!ok) break;
         tc_fence_after();
+        uint32_t dp[64];
+        tmem_ld32(tDP + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
+        tmem_ld32(tDP + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_wait_ld();
+        uint32_t dsp[32];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t dp[32];
-          tmem_ld32(tDP + lane_off + 64 * x + 32 * c, dp);
-          tmem_wait_ld();
-          uint32_t dsp[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd2);
-            const float2 ds = __fmul2_rn(make_float2(pf[32 * c + 2 * i], pf[32 * c + 2 * i + 1]), d2);
-            dsp[i] = pack_bf16(ds.x, ds.y);
-          }
-          // dS pairs of key columns [32c, 32c + 32) -> S columns 64x + [16c, 16c + 16), already read
-          tmem_st16(tS + lane_off + 64 * x + 16 * c, dsp);
+        for (int i = 0; i < 32; ++i) {
+          const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd2);
+          const float2 pv = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u));
+          const float2 ds = __fmul2_rn(pv, d2);
+          dsp[i] = pack_bf16(ds.x, ds.y);
         }
+        // dS pairs of key columns [64x, 64x + 64) -> S columns 64x + [0, 32), already read
+        tmem_st16(tS + lane_off + 64 * x, *reinterpret_cast<const uint32_t(*)[16]>(&dsp[0]));
+        tmem_st16(tS + lane_off + 64 * x + 16, *reinterpret_cast<const uint32_t(*)[16]>(&dsp[16]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(DS_READY));
