@@ -160,6 +160,14 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
                     int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
                     void* workspace, size_t workspace_bytes, int stages, void* stream);
 
+/* Process-wide options.  S2_OPT_FWD_PAIRS (value 0 or 1, default 0): run
+ * the forward of D = 128 without documents on pairs of CTAs whose tensor-core
+ * products span both (tcgen05 cta_group::2, M = 256 rows), halving the shared-
+ * memory operand traffic per product; results equal the single-CTA forward
+ * within rounding.  Not synchronised: set it before launching work. */
+enum { S2_OPT_FWD_PAIRS = 1 };
+int s2attn_set_option(int option, int value);
+
 /* Rotary position prologue ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,
  * "RoPE使用原始位置"): Q and K are rotated at each token's ORIGINAL position
  * ID, never its index inside a group, with position interpolation p -> p·scale
@@ -292,7 +300,7 @@ int s2attn_check_status(void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 106. */
+/* ABI version of this header (major*100 + minor): 107. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

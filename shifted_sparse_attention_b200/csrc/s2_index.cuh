@@ -63,6 +63,8 @@ struct Plan {
   int q_begin;     // rows [0, q_begin) are never queries (a sequence-parallel halo)
   int k_begin;     // rows [0, k_begin) hold no valid key
   long long ds_head_tiles;  // 128x128 dS tiles per (b, h) in the stored-dS backward
+  int nquad[2];    // CTA-pair forward: units of four query tiles per segment, per class
+  int quad_ranks;  // max over classes of nseg * nquad (CTA-pair forward: clusters per head)
   float scale_log2;  // log2(e) / sqrt(D)
   // Packed sequences: per-position document bounds [B, N, 2] = {first position,
   // one past the last position} of the position's document (original
@@ -349,6 +351,9 @@ inline void finish_plan(Plan& p) {
     p.nunit[c] = (nt + 1) / 2;
     p.ntile[c] = nt;
   }
+  for (int c = 0; c < 2; ++c) p.nquad[c] = (p.ntile[c] + 3) / 4;
+  const int q0 = p.nseg[0] * p.nquad[0], q1 = p.nseg[1] * p.nquad[1];
+  p.quad_ranks = q0 > q1 ? q0 : q1;
   const int r0 = p.nseg[0] * p.nunit[0], r1 = p.nseg[1] * p.nunit[1];
   p.ranks = r0 > r1 ? r0 : r1;
   const int k0 = p.nseg[0] * p.ntile[0], k1 = p.nseg[1] * p.ntile[1];

@@ -15,6 +15,7 @@ struct FwdArgs {
   const CUtensorMap* tmK;
   const CUtensorMap* tmV;
   const CUtensorMap* tmO;
+  const CUtensorMap* tmK64;  // k in boxes of 64 rows (CTA-pair forward), or null
   Plan plan;
   float* lse;
   int* status;
@@ -41,6 +42,8 @@ struct BwdArgs {
 };
 
 int launch_fwd(const FwdArgs& a);
+// CTA-pair forward (D = 128, no documents); needs a.tmK64 (boxes of 64 rows of k).
+int launch_fwd_pair(const FwdArgs& a);
 // stages: 1 = prepare (Delta, lse2), 2 = dK/dV pass, 4 = dQ pass; with 8 the
 // dK/dV pass also stores dS and the dQ pass reads it instead of recomputing.
 int launch_bwd(const BwdArgs& a, int stages);

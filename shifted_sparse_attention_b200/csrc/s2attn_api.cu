@@ -92,6 +92,9 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// S2_OPT_FWD_PAIRS: forward over CTA pairs where it applies (process-wide).
+int g_fwd_pairs = 0;
+
 // Shape rules of the method plus the kernels' own support limits.
 int validate(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant) {
   if (variant < S2_STRICT || variant > S2_DENSE_CAUSAL)
@@ -115,11 +118,12 @@ int validate(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_va
   return S2_OK;
 }
 
-int make_tmap(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t H, int64_t D) {
-  // [B*N, H, D] bf16 viewed as a 3-D tensor (D innermost); box = 64 columns x 1 head x 128 rows.
+int make_tmap(DeviceState* st, CUtensorMap* m, const void* base, int64_t B, int64_t N, int64_t H, int64_t D,
+              int box_rows = s2::kTile) {
+  // [B*N, H, D] bf16 viewed as a 3-D tensor (D innermost); box = 64 columns x 1 head x box_rows rows.
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)(B * N)};
   cuuint64_t strides[2] = {(cuuint64_t)(D * 2), (cuuint64_t)(H * D * 2)};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)s2::kTile};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t elem[3] = {1, 1, 1};
   CUresult r = st->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                           elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -150,7 +154,15 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 106; }
+int s2attn_version(void) { return 107; }
+
+int s2attn_set_option(int option, int value) {
+  if (option == S2_OPT_FWD_PAIRS) {
+    g_fwd_pairs = value != 0;
+    return S2_OK;
+  }
+  return fail(S2_ERR_INVALID_ARG, "unknown option %d", option);
+}
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -170,10 +182,17 @@ static int fwd_launch(const void* q, const void* k, const void* v, void* o, floa
     return rc;
   s2::FwdArgs a;
   a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmO = &to;
+  a.tmK64 = nullptr;
   a.plan = plan;
   a.lse = lse;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
+  if (g_fwd_pairs && D == 128 && plan.docs == nullptr) {
+    CUtensorMap tk64;
+    if ((rc = make_tmap(st, &tk64, k, B, N, H, D, 64))) return rc;
+    a.tmK64 = &tk64;
+    return launch_status(s2::launch_fwd_pair(a), "forward (CTA pairs)");
+  }
   return launch_status(s2::launch_fwd(a), "forward");
 }
 
