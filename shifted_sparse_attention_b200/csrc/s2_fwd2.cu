@@ -258,7 +258,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
+    // Nothing is loaded for a cluster without a valid row: no MMA would consume the
+    // loads, and a CTA must not retire with copies into its shared memory in flight.
+    if (lane == 0 && u.kmax >= 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK64);
       prefetch_tmap(&tmV);
