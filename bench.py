@@ -49,6 +49,8 @@ def parse():
                     help="pack documents of this many tokens (document mask); reports exact-pair TFLOP/s")
     ap.add_argument("--sp-emulate", type=int, default=0, metavar="W",
                     help="sequence parallelism: run W ranks' shards (halo exchange + rank kernels) in turn on this GPU")
+    ap.add_argument("--fwd-pairs", type=int, default=None, choices=[0, 1],
+                    help="forward over CTA pairs (tcgen05 cta_group::2) on or off")
     ap.add_argument("--recompute-dq", action="store_true",
                     help="dQ pass recomputes S and dP (8 MB workspace) instead of reading the stored dS")
     ap.add_argument("--rope", action="store_true",
@@ -332,6 +334,8 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
+    if args.fwd_pairs is not None:
+        s2.set_fwd_pairs(bool(args.fwd_pairs))
     w = synthetic.WORKLOADS[args.workload]
     variant = w.variants[0] if args.variant is None else args.variant
     B, N, H, D, G = w.B, w.N, w.H, w.D, w.G
