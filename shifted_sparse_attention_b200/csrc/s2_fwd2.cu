@@ -22,7 +22,7 @@
 // all MMAs.  Handshakes:
 //   K/V, Q loads of both CTAs complete on CTA 0's barriers (.cta_group::2
 //     TMA; CTA 0's producer announces the bytes of both halves);
-//   P_FULL: all 256 softmax threads of the pair arrive on CTA 0's barrier;
+//   P_FULL: each of the pair's 16 softmax warps arrives once on CTA 0's barrier;
 //   S_FULL, KV_EMPTY, MMA_DONE: tcgen05.commit multicast to both CTAs;
 //   EXIT: each CTA tells the other it has read its accumulators, before the
 //     paired TMEM allocation is released.
@@ -234,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(S_FULL + x), 1);
-      mbar_init(bar(P_FULL + x), 256);
+      mbar_init(bar(P_FULL + x), 16);
     }
     mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(MMA_DONE), 1);
@@ -402,8 +402,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + x * 128;
     const uint32_t tO = tmem + lane_off + 256 + x * D;
-    const int tx = u.t[x];
-    const bool px = q.own[x];
+    // scalars: indexing the unit's arrays with the runtime x would move them to local memory
+    const int tx = x ? u.t[1] : u.t[0];
+    const bool px = x ? q.own[1] : q.own[0];
+    const bool pairx = x ? q.pair[1] : q.pair[0];
+    const int kmaxx = x ? q.kmax[1] : q.kmax[0];
     const bool exists = tx < u.ntiles;
     const int q0 = exists ? tile_orig(p, u, tx) : 0;
     const bool row_valid = exists && (q0 + r) < p.n_valid;
@@ -411,8 +414,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
     float m_used = -INFINITY, l = 0.f;
     int n = 0, nt = 0;  // key tiles of the pair / of them this tile takes
     bool ok = true;
-    if (q.pair[x]) {
-      for (int k = 0; k <= q.kmax[x] && ok; ++k) {
+    if (pairx) {
+      for (int k = 0; k <= kmaxx && ok; ++k) {
         if (!ktile_valid(p, u, k)) continue;
         ok = s2_wait_cl(bar(S_FULL + x), n & 1, abort_flag, status, 4);
         if (!ok) break;
@@ -479,7 +482,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
         tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive_cluster(p_full);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(p_full);  // one arrival per warp: 16 per pair
         ++n;
       }
     }
