@@ -22,7 +22,8 @@
 // all MMAs.  Handshakes:
 //   K/V, Q loads of both CTAs complete on CTA 0's barriers (.cta_group::2
 //     TMA; CTA 0's producer announces the bytes of both halves);
-//   P_FULL: each of the pair's 16 softmax warps arrives once on CTA 0's barrier;
+//   P_FULL(x): each of the pair's 8 warps of softmax warpgroup x arrives once on
+//     CTA 0's barrier;
 //   S_FULL, KV_EMPTY, MMA_DONE: tcgen05.commit multicast to both CTAs;
 //   EXIT: each CTA tells the other it has read its accumulators, before the
 //     paired TMEM allocation is released.
@@ -95,9 +96,15 @@ __device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) 
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ void st_cluster_u32(uint32_t cl_addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cl_addr), "r"(v) : "memory");
+}
 // Bounded wait with cluster-scope acquire (arrivals may come from the peer CTA).
+// A timeout sets the abort flag of both CTAs (peer_abort: the peer's flag, as a
+// shared::cluster address), so that every role of the pair gives up promptly and
+// both reach the exit handshake.
 __device__ __forceinline__ bool s2_wait_cl(uint32_t bar, uint32_t parity, volatile int* abort, int* status,
-                                           int code) {
+                                           int code, uint32_t peer_abort) {
   if (mbar_try_wait_cl(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
@@ -105,8 +112,21 @@ __device__ __forceinline__ bool s2_wait_cl(uint32_t bar, uint32_t parity, volati
     if (*abort) return false;
     if (clock64() - t0 > kWaitBudgetCycles) {
       *abort = 1;
+      st_cluster_u32(peer_abort, 1u);
       atomicOr(status, code);
       return false;
+    }
+  }
+}
+// The exit handshake's wait ignores the abort flag: a CTA must not retire while
+// its peer may still reach its shared memory.  Its budget covers the peer's
+// longest way there (one timed-out wait, the others cut short by the flag).
+__device__ __forceinline__ void wait_exit(uint32_t bar, int* status) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait_cl(bar, 0)) {
+    if (clock64() - t0 > 4 * kWaitBudgetCycles) {
+      atomicOr(status, 64);
+      return;
     }
   }
 }
@@ -234,7 +254,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(S_FULL + x), 1);
-      mbar_init(bar(P_FULL + x), 16);
+      mbar_init(bar(P_FULL + x), 8);  // the four warps of warpgroup x in each CTA
     }
     mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(MMA_DONE), 1);
@@ -255,6 +275,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int row_base = u.b * p.N;
   const bool leader = rank == 0;
+  const uint32_t peer_abort = map_to(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
 
   if (warp == 8) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -281,7 +302,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
       // one half tile per load: K rows [64·rank, +64) (both column chunks) or V columns [64·rank, +64)
       auto load = [&](bool isK, int k) {
         const int slot = e % kSlots;
-        if (e >= kSlots) ok = s2_wait_cl(bar(KV_EMPTY + slot), ((e / kSlots) - 1) & 1, abort_flag, status, 1);
+        if (e >= kSlots) ok = s2_wait_cl(bar(KV_EMPTY + slot), ((e / kSlots) - 1) & 1, abort_flag, status, 1, peer_abort);
         if (!ok) return;
         if (leader) mbar_arrive_expect_tx(bar(KV_FULL + slot), 2 * kHalfBytes);
         const uint32_t full = map_to(bar(KV_FULL + slot), 0);
@@ -330,13 +351,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
                    idesc_pv, ((acc) || kk > 0) ? 1u : 0u);                                        \
     }                                                                                             \
   } while (0)
-      bool ok = s2_wait_cl(bar(Q_FULL), 0, abort_flag, status, 2);
+      bool ok = s2_wait_cl(bar(Q_FULL), 0, abort_flag, status, 2, peer_abort);
       int npvA = 0, npvB = 0;
       int e = 0;
       int kc = next_key(p, q, -1);
       if (ok && kc >= 0) {
         const int eK = e++;
-        ok = s2_wait_cl(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
+        ok = s2_wait_cl(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2, peer_abort);
         tc_fence_after();
         if (ok && pair_takes(q, 0, kc)) {
           ISSUE_QK(0, eK % kSlots);
@@ -351,12 +372,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
       int kn = kc >= 0 ? next_key(p, q, kc) : -1;
       int eV = e++;
       int eK = kn >= 0 ? e++ : -1;
-      if (ok && kc >= 0) ok = s2_wait_cl(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2);
-      if (ok && kn >= 0) ok = s2_wait_cl(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2);
+      if (ok && kc >= 0) ok = s2_wait_cl(bar(KV_FULL + eV % kSlots), (eV / kSlots) & 1, abort_flag, status, 2, peer_abort);
+      if (ok && kn >= 0) ok = s2_wait_cl(bar(KV_FULL + eK % kSlots), (eK / kSlots) & 1, abort_flag, status, 2, peer_abort);
       while (ok && kc >= 0) {
         const int sV = eV % kSlots, sK = eK >= 0 ? eK % kSlots : 0;
         if (pair_takes(q, 0, kc)) {
-          ok = s2_wait_cl(bar(P_FULL + 0), npvA & 1, abort_flag, status, 2);
+          ok = s2_wait_cl(bar(P_FULL + 0), npvA & 1, abort_flag, status, 2, peer_abort);
           if (!ok) break;
           tc_fence_after();
           ISSUE_PV(0, sV, npvA > 0);
@@ -369,11 +390,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
         const int knn = kn >= 0 ? next_key(p, q, kn) : -1;
         const int eV2 = kn >= 0 ? e++ : -1;
         const int eK2 = knn >= 0 ? e++ : -1;
-        if (eV2 >= 0) ok = s2_wait_cl(bar(KV_FULL + eV2 % kSlots), (eV2 / kSlots) & 1, abort_flag, status, 2);
-        if (ok && eK2 >= 0) ok = s2_wait_cl(bar(KV_FULL + eK2 % kSlots), (eK2 / kSlots) & 1, abort_flag, status, 2);
+        if (eV2 >= 0) ok = s2_wait_cl(bar(KV_FULL + eV2 % kSlots), (eV2 / kSlots) & 1, abort_flag, status, 2, peer_abort);
+        if (ok && eK2 >= 0) ok = s2_wait_cl(bar(KV_FULL + eK2 % kSlots), (eK2 / kSlots) & 1, abort_flag, status, 2, peer_abort);
         if (!ok) break;
         if (pair_takes(q, 1, kc)) {
-          ok = s2_wait_cl(bar(P_FULL + 1), npvB & 1, abort_flag, status, 2);
+          ok = s2_wait_cl(bar(P_FULL + 1), npvB & 1, abort_flag, status, 2, peer_abort);
           if (!ok) break;
           tc_fence_after();
           ISSUE_PV(1, sV, npvB > 0);
@@ -417,7 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
     if (pairx) {
       for (int k = 0; k <= kmaxx && ok; ++k) {
         if (!ktile_valid(p, u, k)) continue;
-        ok = s2_wait_cl(bar(S_FULL + x), n & 1, abort_flag, status, 4);
+        ok = s2_wait_cl(bar(S_FULL + x), n & 1, abort_flag, status, 4, peer_abort);
         if (!ok) break;
         tc_fence_after();
         uint32_t s[kTile];
@@ -483,13 +504,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(p_full);  // one arrival per warp: 16 per pair
+        if (lane == 0) mbar_arrive_cluster(p_full);  // one arrival per warp: 8 per pair and tile
         ++n;
       }
     }
     // every MMA of the pair has completed (commit multicast to both CTAs)
     if (ok && u.kmax >= 0) {
-      ok = s2_wait_cl(bar(MMA_DONE), 0, abort_flag, status, 4);
+      ok = s2_wait_cl(bar(MMA_DONE), 0, abort_flag, status, 4, peer_abort);
       tc_fence_after();
     }
     // ---------------------------------------------------------- epilogue
@@ -536,7 +557,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
   __syncthreads();
   if (threadIdx.x == 0) {
     mbar_arrive_cluster(map_to(bar(EXIT), rank ^ 1u));
-    s2_wait_cl(bar(EXIT), 0, abort_flag, status, 64);
+    wait_exit(bar(EXIT), status);
   }
   __syncthreads();
   if (warp == 9) {
