@@ -96,66 +96,43 @@ __device__ __forceinline__ void acc_to_smem(uint32_t tacc, uint32_t lane_off, in
 }  // namespace bwd
 
 // ------------------------------------------------------------------ preprocess
-// kTpr = D/8 threads per (b, i, h) row, 8 bf16 (16 bytes) each; a block covers
-// kRows rows, each thread kRep of them (all its loads in flight before the
-// first sum: the pass is a stream of o and dout).  Stores the negated
-// statistics the passes add: -Delta = -(dout·o) and -lse·log2(e) (-inf on rows
-// that are not queries: padding, or a sequence-parallel halo).
-namespace pre {
-constexpr int kThreads = 256, kRep = 4;
+// kTpr = D/8 threads per (b, i, h) row, 8 bf16 (16 bytes) each.  Stores the
+// negated statistics the passes add: -Delta = -(dout·o) and -lse·log2(e)
+// (-inf on padded rows, which zeroes their probabilities).
 template <int D>
-struct Shape {
-  static constexpr int kTpr = D / 8;
-  static constexpr int kRowsPerPass = kThreads / kTpr;
-  static constexpr int kRows = kRowsPerPass * kRep;
-};
-}  // namespace pre
-
-template <int D>
-__global__ void __launch_bounds__(pre::kThreads) s2_bwd_pre(const __nv_bfloat16* __restrict__ o,
-                                                            const __nv_bfloat16* __restrict__ dout,
-                                                            const float* __restrict__ lse, float* __restrict__ delta,
-                                                            float* __restrict__ lse2, int B, int N, int H,
-                                                            int q_begin, int n_valid) {
-  using S = pre::Shape<D>;
-  const int sub = threadIdx.x % S::kTpr;
+__global__ void __launch_bounds__(256) s2_bwd_pre(const __nv_bfloat16* __restrict__ o,
+                                                   const __nv_bfloat16* __restrict__ dout,
+                                                   const float* __restrict__ lse, float* __restrict__ delta,
+                                                   float* __restrict__ lse2, int B, int N, int H, int q_begin,
+                                                   int n_valid) {
+  constexpr int kTpr = D / 8;
+  constexpr int kRowsPerBlock = 256 / kTpr;
+  const long long row = (long long)blockIdx.x * kRowsPerBlock + threadIdx.x / kTpr;
+  const int sub = threadIdx.x % kTpr;
   const long long rows = (long long)B * N * H;
-  const long long base = (long long)blockIdx.x * S::kRows + threadIdx.x / S::kTpr;
-  uint4 a[pre::kRep], g[pre::kRep];
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + row * D + sub * 8);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
 #pragma unroll
-  for (int t = 0; t < pre::kRep; ++t) {
-    const long long row = base + (long long)t * S::kRowsPerPass;
-    if (row < rows) {
-      a[t] = *reinterpret_cast<const uint4*>(o + row * D + sub * 8);
-      g[t] = *reinterpret_cast<const uint4*>(dout + row * D + sub * 8);
-    } else {
-      a[t] = make_uint4(0, 0, 0, 0);
-      g[t] = make_uint4(0, 0, 0, 0);
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < pre::kRep; ++t) {
-    const long long row = base + (long long)t * S::kRowsPerPass;
-    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a[t]);
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g[t]);
-    float acc = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const float2 fa = __bfloat1622float2(a2[c]), fg = __bfloat1622float2(g2[c]);
+    for (int t = 0; t < 4; ++t) {
+      const float2 fa = __bfloat1622float2(a2[t]), fg = __bfloat1622float2(g2[t]);
       acc = fmaf(fa.x, fg.x, acc);
       acc = fmaf(fa.y, fg.y, acc);
     }
+  }
 #pragma unroll
-    for (int off = S::kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, S::kTpr);
-    if (row < rows && sub == 0) {
-      const int h = (int)(row % H);
-      const long long bi = row / H;
-      const int i = (int)(bi % N), b = (int)(bi / N);
-      const size_t at = ((size_t)b * H + h) * N + i;
-      const bool valid = i >= q_begin && i < n_valid;
-      delta[at] = valid ? -acc : 0.f;
-      lse2[at] = valid ? -lse[at] * 1.4426950408889634f : -INFINITY;
-    }
+  for (int off = kTpr / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off, kTpr);
+  if (row < rows && sub == 0) {
+    const int h = (int)(row % H);
+    const long long bi = row / H;
+    const int i = (int)(bi % N), b = (int)(bi / N);
+    const size_t at = ((size_t)b * H + h) * N + i;
+    const bool valid = i >= q_begin && i < n_valid;
+    delta[at] = valid ? -acc : 0.f;
+    lse2[at] = valid ? -lse[at] * 1.4426950408889634f : -INFINITY;
   }
 }
 
@@ -1027,8 +1004,8 @@ int launch_bwd_impl(const BwdArgs& a, int stages) {
   const long long rows = (long long)p.B * p.N * p.H;
   cudaError_t e;
   if (stages & 1) {  // prepare: -Delta and -lse·log2(e)
-    constexpr int kRowsPerBlock = pre::Shape<D>::kRows;
-    s2_bwd_pre<D><<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), pre::kThreads, 0, a.stream>>>(
+    constexpr int kRowsPerBlock = 256 / (D / 8);
+    s2_bwd_pre<D><<<(unsigned)((rows + kRowsPerBlock - 1) / kRowsPerBlock), 256, 0, a.stream>>>(
         static_cast<const __nv_bfloat16*>(a.o), static_cast<const __nv_bfloat16*>(a.dout), a.lse, a.delta, a.lse2,
         p.B, p.N, p.H, p.q_begin, p.n_valid);
     e = cudaGetLastError();
