@@ -24,7 +24,7 @@
 //     TMA; CTA 0's producer announces the bytes of both halves);
 //   P_FULL(x): each of the pair's 8 warps of softmax warpgroup x arrives once on
 //     CTA 0's barrier;
-//   S_FULL, KV_EMPTY, MMA_DONE: tcgen05.commit multicast to both CTAs;
+//   S_FULL, KV_EMPTY, MMA_DONE: tcgen05.commit to the barrier of each CTA;
 //   EXIT: each CTA tells the other it has read its accumulators, before the
 //     paired TMEM allocation is released.
 // Every wait is bounded (s2_wait / s2_wait_cl).  No TMA load uses multicast.
@@ -166,13 +166,15 @@ __device__ __forceinline__ void umma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, u
       "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
-// Arrive on barrier `bar` (same offset) of both CTAs once the issued MMAs complete.
+// Arrive on barrier `bar` (same offset) of both CTAs once the issued MMAs
+// complete: one commit per CTA, the peer's barrier named by its cluster address.
+__device__ __forceinline__ void umma_commit_to(uint32_t cl_bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(cl_bar)
+               : "memory");
+}
 __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
-  asm volatile(
-      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
-          bar)
-      : "memory");
+  umma_commit_to(map_to(bar, 0));
+  umma_commit_to(map_to(bar, 1));
 }
 
 // A cluster's work: four consecutive query tiles of one segment.
@@ -508,7 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(fwd2::kThreads, 1)
         ++n;
       }
     }
-    // every MMA of the pair has completed (commit multicast to both CTAs)
+    // every MMA of the pair has completed (committed to both CTAs)
     if (ok && u.kmax >= 0) {
       ok = s2_wait_cl(bar(MMA_DONE), 0, abort_flag, status, 4, peer_abort);
       tc_fence_after();
