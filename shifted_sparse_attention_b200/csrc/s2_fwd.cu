@@ -51,8 +51,7 @@ enum Bar {
   P_FULL = 12,      // + tile (2)
   Q_FULL = 14,
   MMA_DONE = 15,
-  TURN = 16,        // + tile (2): the other softmax warpgroup has finished its exponentials
-  NUM_BARS = 18
+  NUM_BARS = 16
 };
 
 template <int D>
@@ -138,7 +137,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(bar(S_FULL + x), 1);
       mbar_init(bar(P_FULL + x), 128);
-      mbar_init(bar(TURN + x), 128);
     }
     mbar_init(bar(Q_FULL), 1);
     mbar_init(bar(MMA_DONE), 1);
@@ -310,20 +308,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
       float m_used = -INFINITY, l = 0.f;
       int n = 0;
       bool ok = true;
-      // Without documents the two warpgroups take turns at their exponentials (A, B,
-      // A, B, ... in the MMA order), so that they do not share the MUFU units of an
-      // SM sub-partition and each tile's P is ready sooner.  Both walk the valid key
-      // tiles from the segment start, so their n-th tiles coincide while both have
-      // one; n_other: the key tiles of the other warpgroup, i.e. its turns.  (Under
-      // a document mask the two sequences differ and no turns are taken.)
-      int n_other = 0;
-      if constexpr (!kDocs) {
-        const int to = x ? tA : tB;
-        const bool po = x ? pA : pB;
-        if (po && to >= 0)
-          for (int k = 0; k <= to; ++k)
-            if (ktile_valid(p, u, k)) ++n_other;
-      }
       if (px) {
         for (int k = 0; k <= tx && ok; ++k) {
           if (!ktile_valid(p, u, k) || (kDocs && !tile_meets(tile_orig(p, u, k), lx, hx))) continue;
@@ -371,12 +355,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           // accumulators, so o = sum p~ v / sum p~ stays a convex combination of the v_j.
           const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
           const float2 nm2 = make_float2(-m_exp, -m_exp);
-          // my turn: A's n-th exponentials follow B's (n-1)-th, B's n-th follow A's n-th
-          if (!kDocs && (x == 0 ? (n >= 1 && n - 1 < n_other) : (n < n_other))) {
-            const int idx = x == 0 ? n - 1 : n;
-            ok = s2_wait(bar(TURN + x), idx & 1, abort_flag, status, 4);
-            if (!ok) break;
-          }
           float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
           for (int c = 0; c < kTile; c += 2) {
@@ -385,7 +363,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             s[c / 2] = pk;
             acc[(c / 2) & 3] = __fadd2_rn(acc[(c / 2) & 3], make_float2(__uint_as_float(pk << 16), __uint_as_float(pk & 0xffff0000u)));
           }
-          if constexpr (!kDocs) mbar_arrive(bar(TURN + (1 - x)));  // the other warpgroup's turn
           const float2 acc01 = __fadd2_rn(acc[0], acc[1]), acc23 = __fadd2_rn(acc[2], acc[3]);
           const float2 acct = __fadd2_rn(acc01, acc23);
           l += acct.x + acct.y;
