@@ -352,3 +352,24 @@ def test_stored_ds_workspace_size(abi):
     ws = L.s2attn_bwd_ds_workspace_size(1, 1024, 8, 64, 256, 0)
     rc = L.s2attn_bwd_stages_v(*([fake] * 9), 1, 1024, 8, 64, 256, 1024, 0, fake, ws - 1, 15, None)
     assert rc == abi.S2_ERR_INVALID_ARG  # workspace too small for the stored dS
+
+
+def test_bench_tile_pair_count_matches_the_kernels_traversal(harness):
+    # bench.py prices the stored-dS dQ pass on a closed count of tile pairs; it must
+    # equal the number of dS tiles the kernels' traversal writes
+    import bench
+    from types import SimpleNamespace
+
+    for (N, G, nv, variant) in [(1024, 256, 1024, 0), (1536, 512, 1400, 0), (2048, 512, 2048, 1),
+                                (2048, 1024, 1700, 1), (1024, 1024, 900, 2)]:
+        B, H = 1, 2
+        d = None
+        total = B * H * _ds_head_tiles(N, G, variant)
+        w = np.zeros(total, dtype=np.int32)
+        r = np.zeros(total, dtype=np.int32)
+        harness.s2h_ds_slots(B, N, H, G, nv, variant, d, w.ctypes.data, r.ctypes.data)
+        wl = SimpleNamespace(N=N, G=G, valid=nv)
+        counted = sum(bench.stored_tile_pairs(wl, variant, c) for c in ((0,) if variant == 2 else (0, 1)))
+        if variant == 2:
+            counted *= 2  # both heads of the dense graph are class 0
+        assert int(w.sum()) == counted, (N, G, nv, variant, int(w.sum()), counted)
