@@ -260,6 +260,14 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           ISSUE_QK(0, sK);
           umma_commit(bar(S_FULL + 0));
         }
+        // The next iteration's tile and loads, while tile A's products are queued:
+        // the issuing thread's bookkeeping then never leaves the tensor core idle.
+        const int knn = kn >= 0 ? NEXT_K(kn) : -1;
+        const int eV2 = kn >= 0 ? e++ : -1;   // V(kn)
+        const int eK2 = knn >= 0 ? e++ : -1;  // K(knn)
+        if (eV2 >= 0) ok = s2_wait(bar(KV_FULL + eV2 % kSlots), (eV2 / kSlots) & 1, abort_flag, status, 2);
+        if (ok && eK2 >= 0) ok = s2_wait(bar(KV_FULL + eK2 % kSlots), (eK2 / kSlots) & 1, abort_flag, status, 2);
+        if (!ok) break;
         if (TAKES_B(kc)) {
           ok = s2_wait(bar(P_FULL + 1), npvB & 1, abort_flag, status, 2);
           if (!ok) break;
@@ -273,15 +281,6 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
         umma_commit(bar(KV_EMPTY + sV));
         if (kn >= 0) umma_commit(bar(KV_EMPTY + sK));
-        // The next iteration's loads, waited for behind both tiles' products: a late
-        // tile then costs no issue slot of this iteration, and the pipe has tile B's
-        // products to work on meanwhile.
-        const int knn = kn >= 0 ? NEXT_K(kn) : -1;
-        const int eV2 = kn >= 0 ? e++ : -1;   // V(kn)
-        const int eK2 = knn >= 0 ? e++ : -1;  // K(knn)
-        if (eV2 >= 0) ok = s2_wait(bar(KV_FULL + eV2 % kSlots), (eV2 / kSlots) & 1, abort_flag, status, 2);
-        if (ok && eK2 >= 0) ok = s2_wait(bar(KV_FULL + eK2 % kSlots), (eK2 / kSlots) & 1, abort_flag, status, 2);
-        if (!ok) break;
         kc = kn;
         kn = knn;
         eV = eV2;
