@@ -9,7 +9,10 @@
 // delivers 6 KB instead of 8 KB, per key tile a CTA loads 32 KB of K/V
 // instead of 64 KB, and one thread issues the MMAs for both CTAs: the score
 // MMAs of the single-CTA kernel, with both operands in shared memory, run at
-// the SM's shared-memory bandwidth, which this layout relieves.
+// the SM's shared-memory bandwidth, which this layout relieves.  Measured on the
+// long-context workload it is nevertheless slower (2.97 against 2.25 ms): a
+// pair product still takes 72-79 cycles to issue, and each tile's hand-off now
+// waits for the slower softmax of two CTAs.  It is an option, off by default.
 //
 // A cluster of two CTAs owns four consecutive 128-row query tiles of one
 // segment: CTA r holds tiles A = 4w + r and B = 4w + 2 + r, so the "A pair"
