@@ -297,10 +297,18 @@ int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, i
  * on the current device since the last check: S2_OK or S2_ERR_TIMEOUT. */
 int s2attn_check_status(void* stream);
 
+/* Failure-detection probe: launches one CTA whose wait on a barrier that
+ * nothing completes runs out after `budget_cycles` SM clocks (in [1000, 4e9]);
+ * the kernel records the timeout in the status word (flag 0x200) and exits
+ * normally, so the next s2attn_check_status() returns S2_ERR_TIMEOUT and the
+ * context stays usable.  It exercises, without any fault, the path every
+ * kernel takes when one of its bounded waits gives up. */
+int s2attn_debug_wait_probe(int64_t budget_cycles, void* stream);
+
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 107. */
+/* ABI version of this header (major*100 + minor): 108. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

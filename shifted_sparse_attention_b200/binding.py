@@ -48,6 +48,7 @@ SIGNATURES = {
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
     "s2attn_set_option": ([_int, _int], _int),
+    "s2attn_debug_wait_probe": ([_i64, _vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
     "s2attn_version": ([], _int),
 }
@@ -345,6 +346,10 @@ def debug_adjacency(N: int, G: int, variant: int, head_class: int, n_valid: int 
         out = torch.empty((N, 4), dtype=torch.int32, device=device)
     _check(s2attn_debug_adjacency(N, G, nv, variant, head_class, fmt, out))
     return out
+
+
+def s2attn_debug_wait_probe(budget_cycles, stream=None) -> int:
+    return lib().s2attn_debug_wait_probe(budget_cycles, _stream(stream))
 
 
 def check_status(stream=None) -> None:

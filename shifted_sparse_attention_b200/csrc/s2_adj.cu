@@ -11,6 +11,7 @@
 
 #include "s2_index.cuh"
 #include "s2_kernels.h"
+#include "sm100_ptx.cuh"
 
 namespace s2 {
 
@@ -69,6 +70,42 @@ int launch_adjacency(const Plan& p0, int head_class, int format, void* out, cuda
   const int grid = grid_fwd(p);
   s2_adjacency_kernel<<<grid, 256, 0, stream>>>(p, head_class, format, static_cast<uint32_t*>(out),
                                                 static_cast<int*>(out));
+  return (int)cudaGetLastError();
+}
+
+// Failure-detection probe: the kernels' bounded-wait path, exercised without a
+// fault.  Two warps of one CTA wait on an mbarrier that nothing completes:
+// warp 0 with a short clock budget -- it gives up, raises the CTA's abort flag
+// and records bit 512 in the status word, as a kernel role does on a timeout;
+// warp 1 with the kernels' own bounded wait, which returns as soon as the flag
+// is up.  The CTA then exits normally and the context stays usable.
+__global__ void s2_wait_probe_kernel(int* __restrict__ status, long long budget) {
+  __shared__ alignas(8) uint64_t bar_word;
+  __shared__ int abort_word;
+  const uint32_t b = smem_u32(&bar_word);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_word = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(b, 0)) {
+      if (clock64() - t0 > budget) {
+        *reinterpret_cast<volatile int*>(&abort_word) = 1;
+        atomicOr(status, 512);
+        break;
+      }
+    }
+  } else if (threadIdx.x == 32) {
+    s2_wait(b, 0, reinterpret_cast<volatile int*>(&abort_word), status, 1024);
+  }
+  __syncthreads();
+}
+
+int launch_wait_probe(int* status, long long budget, cudaStream_t stream) {
+  s2_wait_probe_kernel<<<1, 64, 0, stream>>>(status, budget);
   return (int)cudaGetLastError();
 }
 

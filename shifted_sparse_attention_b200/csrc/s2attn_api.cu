@@ -154,7 +154,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 107; }
+int s2attn_version(void) { return 108; }
 
 int s2attn_set_option(int option, int value) {
   if (option == S2_OPT_FWD_PAIRS) {
@@ -478,6 +478,16 @@ int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, i
   s2::Plan p = s2::make_plan(1, (int)N, 2, 128, (int)G, (int)n_valid, variant);
   const int cls = (variant == S2_DENSE_CAUSAL) ? 0 : head_class;
   return launch_status(s2::launch_adjacency(p, cls, format, out, static_cast<cudaStream_t>(stream)), "adjacency");
+}
+
+int s2attn_debug_wait_probe(int64_t budget_cycles, void* stream) {
+  if (budget_cycles < 1000 || budget_cycles > 4000000000LL)
+    return fail(S2_ERR_INVALID_ARG, "budget of %lld cycles outside [1000, 4e9]", (long long)budget_cycles);
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  return launch_status(s2::launch_wait_probe(st->status, (long long)budget_cycles, static_cast<cudaStream_t>(stream)),
+                       "wait probe");
 }
 
 int s2attn_check_status(void* stream) {

@@ -173,7 +173,7 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 107
+    assert L.s2attn_version() == 108
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
