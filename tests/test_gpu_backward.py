@@ -36,6 +36,14 @@ CASES = [
     (1, 1536, 4, 128, 768, DENSE, 1409),
     (1, 1536, 2, 128, 768, STRICT, 129),
     (1, 4096, 2, 128, 1024, ROLLED, 3000),
+    # degenerate shapes: a single valid row, one group per sequence (G = N), the
+    # smallest dense sequence, six heads, three batch rows
+    (1, 1024, 2, 128, 256, STRICT, 1),
+    (1, 1024, 2, 128, 256, ROLLED, 1),
+    (1, 256, 2, 64, 256, STRICT, None),
+    (1, 256, 2, 128, 256, ROLLED, 200),
+    (1, 128, 2, 128, 128, DENSE, None),
+    (3, 1024, 6, 64, 512, STRICT, 777),
 ]
 
 

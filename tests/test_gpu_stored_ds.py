@@ -31,6 +31,9 @@ CASES = [
     (1, 1536, 4, 128, 768, DENSE, 1409),
     (1, 1536, 2, 128, 768, STRICT, 129),
     (1, 4096, 4, 128, 1024, STRICT, None),
+    (1, 1024, 2, 128, 256, ROLLED, 1),       # a single valid row
+    (1, 256, 2, 64, 256, STRICT, None),      # one group per sequence
+    (3, 1024, 6, 64, 512, STRICT, 777),
 ]
 
 
