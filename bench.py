@@ -365,16 +365,23 @@ def run_ours(args, rank, world, local_rank):
         if args.doc_len:
             positions = (torch.arange(N, device=dev, dtype=torch.int32) % args.doc_len).expand(B, N).contiguous()
 
+    nvtx = torch.cuda.nvtx  # ranges name each stage on a profiler's timeline
+
     def step(ev=None):
         if args.rope:
             if ev is not None:
                 ev[5].record(stream)
+            nvtx.range_push("s2 rope")
             s2.rope(q, k, positions, scale=0.25, out=(q_in, k_in))
+            nvtx.range_pop()
         if ev is not None:
             ev[0].record(stream)
+        nvtx.range_push("s2 forward")
         s2.forward(q_in, k_in, v, G, variant, nv, out=o, lse=lse, docs=docs)
+        nvtx.range_pop()
         if ev is not None:
             ev[1].record(stream)
+        nvtx.range_push("s2 backward")
         s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_PREPARE,
                     docs=docs, stored_ds=stored)
         if ev is not None:
@@ -385,6 +392,7 @@ def run_ours(args, rank, world, local_rank):
             ev[3].record(stream)
         s2.backward(q_in, k_in, v, o, do, lse, G, variant, nv, grads=grads, workspace=ws, stages=s2.S2_BWD_DQ,
                     docs=docs, stored_ds=stored)
+        nvtx.range_pop()
         if ev is not None:
             ev[4].record(stream)
 
