@@ -233,6 +233,16 @@ int s2attn_sp_bwd(const void* q, const void* k, const void* v, const void* o, co
                   int64_t D, int64_t G, int64_t n_valid, int variant, int rank, int world,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* The rank backward stage by stage, as s2attn_bwd_stages_v (S2_BWD_STORE_DS
+ * included: the workspace must then hold s2attn_sp_ds_workspace_size bytes). */
+int s2attn_sp_bwd_stages(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t L, int64_t H,
+                         int64_t D, int64_t G, int64_t n_valid, int variant, int rank, int world,
+                         void* workspace, size_t workspace_bytes, int stages, void* stream);
+
+size_t s2attn_sp_ds_workspace_size(int64_t B, int64_t L, int64_t H, int64_t D, int64_t G, int variant,
+                                   int rank, int world);
+
 size_t s2attn_sp_halo_bytes(int64_t B, int64_t H, int64_t D, int64_t G);
 
 int s2attn_sp_halo_pack(const void* a, const void* b, void* msg, int64_t B, int64_t L, int64_t H,

@@ -43,6 +43,9 @@ SIGNATURES = {
     "s2attn_sp_bwd": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int, _int,
                        _int, _vp, _sz, _vp], _int),
     "s2attn_sp_halo_bytes": ([_i64, _i64, _i64, _i64], _sz),
+    "s2attn_sp_bwd_stages": ([_vp, _vp, _vp, _vp, _vp, _fp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _i64, _int,
+                              _int, _int, _vp, _sz, _int, _vp], _int),
+    "s2attn_sp_ds_workspace_size": ([_i64, _i64, _i64, _i64, _i64, _int, _int, _int], _sz),
     "s2attn_sp_halo_pack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_sp_halo_unpack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
@@ -220,6 +223,17 @@ def s2attn_sp_bwd(q, k, v, o, dout, lse, dq, dk, dv, B, L, H, D, G, n_valid, var
     return lib().s2attn_sp_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
                                _ptr(dv), B, L, H, D, G, n_valid, variant, rank, world, _ptr(workspace),
                                workspace_bytes, _stream(stream))
+
+
+def s2attn_sp_bwd_stages(q, k, v, o, dout, lse, dq, dk, dv, B, L, H, D, G, n_valid, variant, rank, world, workspace,
+                         workspace_bytes, stages, stream=None) -> int:
+    return lib().s2attn_sp_bwd_stages(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                      _ptr(dv), B, L, H, D, G, n_valid, variant, rank, world, _ptr(workspace),
+                                      workspace_bytes, stages, _stream(stream))
+
+
+def s2attn_sp_ds_workspace_size(B, L, H, D, G, variant, rank, world) -> int:
+    return int(lib().s2attn_sp_ds_workspace_size(B, L, H, D, G, variant, rank, world))
 
 
 def s2attn_sp_halo_bytes(B, H, D, G) -> int:

@@ -391,14 +391,29 @@ int s2attn_sp_fwd(const void* q, const void* k, const void* v, void* o, float* l
   return fwd_launch(q, k, v, o, lse, plan_sp(B, L, H, D, G, n_valid, variant, rank), stream);
 }
 
+int s2attn_sp_bwd_stages(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, void* dq, void* dk, void* dv, int64_t B, int64_t L, int64_t H, int64_t D,
+                         int64_t G, int64_t n_valid, int variant, int rank, int world, void* workspace,
+                         size_t workspace_bytes, int stages, void* stream) {
+  int rc = validate_sp(B, L, H, D, G, n_valid, variant, rank, world);
+  if (rc) return rc;
+  return bwd_launch(q, k, v, o, dout, lse, dq, dk, dv, plan_sp(B, L, H, D, G, n_valid, variant, rank), workspace,
+                    workspace_bytes, stages, stream);
+}
+
 int s2attn_sp_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
                   void* dq, void* dk, void* dv, int64_t B, int64_t L, int64_t H, int64_t D, int64_t G,
                   int64_t n_valid, int variant, int rank, int world, void* workspace, size_t workspace_bytes,
                   void* stream) {
-  int rc = validate_sp(B, L, H, D, G, n_valid, variant, rank, world);
-  if (rc) return rc;
-  return bwd_launch(q, k, v, o, dout, lse, dq, dk, dv, plan_sp(B, L, H, D, G, n_valid, variant, rank), workspace,
-                    workspace_bytes, S2_BWD_ALL, stream);
+  return s2attn_sp_bwd_stages(q, k, v, o, dout, lse, dq, dk, dv, B, L, H, D, G, n_valid, variant, rank, world,
+                              workspace, workspace_bytes, S2_BWD_ALL, stream);
+}
+
+size_t s2attn_sp_ds_workspace_size(int64_t B, int64_t L, int64_t H, int64_t D, int64_t G, int variant, int rank,
+                                   int world) {
+  if (validate_sp(B, L, H, D, G, L, variant, rank, world) != S2_OK) return 0;
+  const s2::Plan p = plan_sp(B, L, H, D, G, L, variant, rank);
+  return s2attn_bwd_workspace_size(B, G / 2 + L, H, D) + ds_bytes(p);
 }
 
 size_t s2attn_sp_halo_bytes(int64_t B, int64_t H, int64_t D, int64_t G) {

@@ -140,20 +140,25 @@ class SequenceParallelS2Attn:
         return o, l
 
     def backward(self, q_ext, k_ext, v_ext, o_ext, dout_ext, lse_ext, n_valid: int | None = None, grads=None,
-                 workspace=None, exchange: bool = True):
+                 workspace=None, exchange: bool = True, stored_ds: bool = False):
         """The rank's backward (k_ext, v_ext still hold the forward's halo), then the
-        halo gradient exchange; returns (dq_ext, dk_ext, dv_ext)."""
+        halo gradient exchange; returns (dq_ext, dk_ext, dv_ext).  stored_ds: the
+        dK/dV stage keeps dS for the dQ stage (see include/s2attn.h)."""
         B, L, H, D = self._dims(q_ext)
         nv = L if n_valid is None else int(n_valid)
         if grads is None:
             grads = (torch.empty_like(q_ext), torch.empty_like(k_ext), torch.empty_like(v_ext))
         dq, dk, dv = grads
-        ws_bytes = s2.s2attn_bwd_workspace_size(B, self.s + L, H, D)
+        if stored_ds:
+            ws_bytes = s2.s2attn_sp_ds_workspace_size(B, L, H, D, self.G, self.variant, self.rank, self.world)
+        else:
+            ws_bytes = s2.s2attn_bwd_workspace_size(B, self.s + L, H, D)
         if workspace is None:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q_ext.device)
-        s2._check(s2.s2attn_sp_bwd(q_ext, k_ext, v_ext, o_ext, dout_ext, lse_ext, dq, dk, dv, B, L, H, D, self.G, nv,
-                                   self.variant, self.rank, self.world, workspace,
-                                   workspace.numel() * workspace.element_size()))
+        stages = s2.S2_BWD_ALL_DS if stored_ds else s2.S2_BWD_ALL
+        s2._check(s2.s2attn_sp_bwd_stages(q_ext, k_ext, v_ext, o_ext, dout_ext, lse_ext, dq, dk, dv, B, L, H, D,
+                                          self.G, nv, self.variant, self.rank, self.world, workspace,
+                                          workspace.numel() * workspace.element_size(), stages))
         if exchange:
             self.exchange_grad(dk, dv)
         return dq, dk, dv

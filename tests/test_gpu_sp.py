@@ -28,7 +28,7 @@ from tests.tolerance import check_grad, check_lse, check_o, to_np
 pytestmark = pytest.mark.gpu
 
 
-def _emulate(x, G, variant, W, nv_last):
+def _emulate(x, G, variant, W, nv_last, stored=False):
     """Run the W ranks in turn; returns global (o, lse, dq, dk, dv)."""
     B, N, H, D = x["q"].shape
     L, s = N // W, G // 2
@@ -55,9 +55,14 @@ def _emulate(x, G, variant, W, nv_last):
         lse = torch.empty((B, H, s + L), dtype=torch.float32, device="cuda")
         s2._check(s2.s2attn_sp_fwd(ext["q"][r], ext["k"][r], ext["v"][r], o, lse, B, L, H, D, G, nv, variant, r, W))
         dq, dk, dv = (torch.empty_like(o) for _ in range(3))
-        ws = torch.empty(s2.s2attn_bwd_workspace_size(B, s + L, H, D), dtype=torch.uint8, device="cuda")
-        s2._check(s2.s2attn_sp_bwd(ext["q"][r], ext["k"][r], ext["v"][r], o, ext["dout"][r], lse, dq, dk, dv, B, L,
-                                   H, D, G, nv, variant, r, W, ws, ws.numel()))
+        if stored:
+            ws = torch.empty(s2.s2attn_sp_ds_workspace_size(B, L, H, D, G, variant, r, W), dtype=torch.uint8,
+                             device="cuda")
+        else:
+            ws = torch.empty(s2.s2attn_bwd_workspace_size(B, s + L, H, D), dtype=torch.uint8, device="cuda")
+        s2._check(s2.s2attn_sp_bwd_stages(ext["q"][r], ext["k"][r], ext["v"][r], o, ext["dout"][r], lse, dq, dk, dv,
+                                          B, L, H, D, G, nv, variant, r, W, ws, ws.numel(),
+                                          s2.S2_BWD_ALL_DS if stored else s2.S2_BWD_ALL))
         outs.append(dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv))
     for r in range(W):  # halo gradients go back to the rank the halo came from
         to, frm = sp.peers(r, W, variant)
@@ -71,10 +76,10 @@ def _emulate(x, G, variant, W, nv_last):
     return cat("o"), lse, cat("dq"), cat("dk"), cat("dv")
 
 
-def _single(x, G, variant, nv):
+def _single(x, G, variant, nv, stored=False):
     dev = {n: t.cuda() for n, t in x.items()}
     o, lse = s2.forward(dev["q"], dev["k"], dev["v"], G, variant, nv)
-    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, G, variant, nv)
+    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, G, variant, nv, stored_ds=stored)
     torch.cuda.synchronize()
     s2.check_status()
     return o, lse, dq, dk, dv
@@ -101,13 +106,14 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("stored", [False, True], ids=["recompute", "stored_ds"])
 @pytest.mark.parametrize("B,H,D,G,W,L,variant,pad", CASES)
-def test_sequence_parallel_matches_single_gpu_and_oracle(B, H, D, G, W, L, variant, pad):
+def test_sequence_parallel_matches_single_gpu_and_oracle(B, H, D, G, W, L, variant, pad, stored):
     N, s = W * L, G // 2
     nv = N - pad
     x = synthetic.draw(B, N, H, D, seed=W * 100 + L + variant)
-    o, lse, dq, dk, dv = _emulate(x, G, variant, W, L - pad)
-    o1, lse1, dq1, dk1, dv1 = _single(x, G, variant, nv)
+    o, lse, dq, dk, dv = _emulate(x, G, variant, W, L - pad, stored)
+    o1, lse1, dq1, dk1, dv1 = _single(x, G, variant, nv, stored)
     assert torch.equal(o, o1)
     assert torch.equal(lse, lse1)
     assert torch.equal(dq, dq1)
