@@ -626,7 +626,9 @@ def run_sp_emulated(args):
         t["o"] = torch.empty_like(t["q"])
         t["lse"] = torch.empty((B, H, s + L), dtype=torch.float32, device="cuda")
         t["g"] = tuple(torch.empty_like(t["q"]) for _ in range(3))
-        t["ws"] = torch.empty(s2.s2attn_bwd_workspace_size(B, s + L, H, D), dtype=torch.uint8, device="cuda")
+        ws_bytes = (s2.s2attn_bwd_workspace_size(B, s + L, H, D) if args.recompute_dq
+                    else s2.s2attn_sp_ds_workspace_size(B, L, H, D, G, variant, r, W))
+        t["ws"] = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
         ranks.append(t)
     del x
     msg = torch.empty((2, B, s, H // 2, D), dtype=torch.bfloat16, device="cuda")
@@ -645,8 +647,9 @@ def run_sp_emulated(args):
             ev[1].record(stream)
         s2._check(s2.s2attn_sp_fwd(t["q"], t["k"], t["v"], t["o"], t["lse"], B, L, H, D, G, L, variant, r, W))
         dq, dk, dv = t["g"]
-        s2._check(s2.s2attn_sp_bwd(t["q"], t["k"], t["v"], t["o"], t["dout"], t["lse"], dq, dk, dv, B, L, H, D, G,
-                                   L, variant, r, W, t["ws"], t["ws"].numel()))
+        s2._check(s2.s2attn_sp_bwd_stages(t["q"], t["k"], t["v"], t["o"], t["dout"], t["lse"], dq, dk, dv, B, L, H,
+                                          D, G, L, variant, r, W, t["ws"], t["ws"].numel(),
+                                          s2.S2_BWD_ALL if args.recompute_dq else s2.S2_BWD_ALL_DS))
         if ev is not None:
             ev[2].record(stream)
         if frm is not None:
@@ -685,7 +688,8 @@ def run_sp_emulated(args):
         "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": dict(_config(w, variant), parallelism="sp%d-emulated" % W, shard_rows=L),
+        "config": dict(_config(w, variant), parallelism="sp%d-emulated" % W, shard_rows=L,
+                       backward="recomputing dQ pass" if args.recompute_dq else "stored dS"),
         "pct_of_peak": {"bf16_burst": value / pk["bf16_burst"], "bf16_sustained": value / pk["bf16_sustained"]},
         "sp": {"world": W, "per_rank_ms": per_rank, "halo_kernels_ms": halo,
                "halo_bytes_per_direction": v_kv,
