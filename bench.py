@@ -51,6 +51,8 @@ def parse():
                     help="sequence parallelism: run W ranks' shards (halo exchange + rank kernels) in turn on this GPU")
     ap.add_argument("--fwd-pairs", type=int, default=None, choices=[0, 1],
                     help="forward over CTA pairs (tcgen05 cta_group::2) on or off")
+    ap.add_argument("--dkdv-half", type=int, default=None, choices=[0, 1],
+                    help="dK/dV pass over half query tiles with double-buffered scores, on or off")
     ap.add_argument("--recompute-dq", action="store_true",
                     help="dQ pass recomputes S and dP (8 MB workspace) instead of reading the stored dS")
     ap.add_argument("--rope", action="store_true",
@@ -336,6 +338,8 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     if args.fwd_pairs is not None:
         s2.set_fwd_pairs(bool(args.fwd_pairs))
+    if args.dkdv_half is not None:
+        s2.set_dkdv_half(bool(args.dkdv_half))
     w = synthetic.WORKLOADS[args.workload]
     variant = w.variants[0] if args.variant is None else args.variant
     B, N, H, D, G = w.B, w.N, w.H, w.D, w.G

@@ -165,7 +165,11 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
  * products span both (tcgen05 cta_group::2, M = 256 rows), halving the shared-
  * memory operand traffic per product; results equal the single-CTA forward
  * within rounding.  Not synchronised: set it before launching work. */
-enum { S2_OPT_FWD_PAIRS = 1 };
+/* S2_OPT_DKDV_HALF (0 or 1, default 0): run the dK/dV pass over half query
+ * tiles of 64 rows with its score regions double-buffered in tensor memory
+ * (the products of the next half overlap the exponentials of the current
+ * one); results equal the default pass within rounding. */
+enum { S2_OPT_FWD_PAIRS = 1, S2_OPT_DKDV_HALF = 2 };
 int s2attn_set_option(int option, int value);
 
 /* Rotary position prologue ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,

@@ -201,11 +201,16 @@ def rope(q, k, positions=None, base: float = 10000.0, scale: float = 1.0, inplac
 
 
 S2_SP_KV, S2_SP_GRAD = 0, 1
-S2_OPT_FWD_PAIRS = 1
+S2_OPT_FWD_PAIRS, S2_OPT_DKDV_HALF = 1, 2
 
 
 def s2attn_set_option(option, value) -> int:
     return lib().s2attn_set_option(option, value)
+
+
+def set_dkdv_half(enabled: bool) -> None:
+    """Run the dK/dV pass over half query tiles (see include/s2attn.h)."""
+    _check(s2attn_set_option(S2_OPT_DKDV_HALF, 1 if enabled else 0))
 
 
 def set_fwd_pairs(enabled: bool) -> None:

@@ -37,6 +37,8 @@ struct BwdArgs {
   float* delta;       // workspace [B, H, N]: -(dout_i·o_i)
   float* lse2;        // workspace [B, H, N]: -lse_i·log2(e), -inf on padded rows
   void* ds;           // stored-dS workspace (bf16 tiles of 32 KB, see s2_index.cuh), or null
+  const CUtensorMap* tmQ64;   // q in boxes of 64 rows: the dK/dV pass over half query tiles, or null
+  const CUtensorMap* tmdO64;  // dout in boxes of 64 rows (with tmQ64)
   int* status;
   cudaStream_t stream;
 };

@@ -94,6 +94,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // S2_OPT_FWD_PAIRS: forward over CTA pairs where it applies (process-wide).
 int g_fwd_pairs = 0;
+// S2_OPT_DKDV_HALF: the dK/dV pass over half query tiles (process-wide).
+int g_dkdv_half = 0;
 
 // Shape rules of the method plus the kernels' own support limits.
 int validate(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant) {
@@ -159,6 +161,10 @@ int s2attn_version(void) { return 108; }
 int s2attn_set_option(int option, int value) {
   if (option == S2_OPT_FWD_PAIRS) {
     g_fwd_pairs = value != 0;
+    return S2_OK;
+  }
+  if (option == S2_OPT_DKDV_HALF) {
+    g_dkdv_half = value != 0;
     return S2_OK;
   }
   return fail(S2_ERR_INVALID_ARG, "unknown option %d", option);
@@ -331,6 +337,15 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
   // stored dS: bf16 tiles of 32 KB after the row statistics (bulk copies need 16-byte alignment)
   a.ds = stored ? static_cast<char*>(workspace) + stats : nullptr;
+  a.tmQ64 = nullptr;
+  a.tmdO64 = nullptr;
+  CUtensorMap tq64, tdo64;
+  if (g_dkdv_half) {
+    if ((rc = make_tmap(st, &tq64, q, B, N, H, D, 64)) || (rc = make_tmap(st, &tdo64, dout, B, N, H, D, 64)))
+      return rc;
+    a.tmQ64 = &tq64;
+    a.tmdO64 = &tdo64;
+  }
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");
