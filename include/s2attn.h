@@ -164,11 +164,15 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
  * the forward of D = 128 without documents on pairs of CTAs whose tensor-core
  * products span both (tcgen05 cta_group::2, M = 256 rows), halving the shared-
  * memory operand traffic per product; results equal the single-CTA forward
- * within rounding.  Not synchronised: set it before launching work. */
+ * within rounding.  Slower than the default on the workloads measured so
+ * far (2.97 against 2.25 ms on B1 H32 N32768 D128 G8192).  Not synchronised:
+ * set it before launching work. */
 /* S2_OPT_DKDV_HALF (0 or 1, default 0): run the dK/dV pass over half query
  * tiles of 64 rows with its score regions double-buffered in tensor memory
  * (the products of the next half overlap the exponentials of the current
- * one); results equal the default pass within rounding. */
+ * one); results equal the default pass within rounding.  Slower than the
+ * default on the workloads measured so far (5.88 against 4.65 ms on
+ * B1 H32 N32768 D128 G8192). */
 enum { S2_OPT_FWD_PAIRS = 1, S2_OPT_DKDV_HALF = 2 };
 int s2attn_set_option(int option, int value);
 
