@@ -16,16 +16,22 @@
 //        S^T = K Q^T, dP^T = V dO^T (TMEM);  P^T = exp2(S^T·c - lse2) and
 //        dS^T = P^T (dP^T - Delta) on the CUDA cores, both written back to
 //        TMEM as bf16;  dV += P^T dO and dK += dS^T Q with A read from TMEM.
-//   3. s2_bwd_dq_kernel: query-major, one CTA per 128-query tile, walking the
-//      key tiles from the segment start to the diagonal:
-//        S = Q K^T, dP = dO V^T (TMEM);  dS = P (dP - Delta) -> TMEM (bf16);
-//        dQ += dS K with A read from TMEM;  dq = bf16(dQ / sqrt(D)).
-// The dq pass recomputes S and dP (two of its three products), so the
-// backward does 7 instead of 5 tile products per (key tile, query tile) pair.
-// In exchange dq is written once, in bf16, without a float32 accumulator:
+//   3. the dq pass, query-major, one CTA per 128-query tile, walking the key
+//      tiles from the segment start to the diagonal, in one of two forms:
+//      - s2_bwd_dq_ds_kernel (stages with S2_BWD_STORE_DS): the dK/dV pass
+//        has also written every dS tile (bf16) to the workspace, and
+//        dQ += dS K streams them back (HBM-bound, no exponentials);
+//      - s2_bwd_dq_kernel: recomputes S = Q K^T and dP = dO V^T (TMEM),
+//        dS = P (dP - Delta) -> TMEM (bf16), dQ += dS K with A from TMEM.
+//      Either way dq = bf16(dQ / sqrt(D)) is written once.
+// The recomputing form does 7 instead of 5 tile products per (key tile,
+// query tile) pair; the stored form trades the two extra products for 32 KB
+// of dS written and read per pair.  Neither needs a float32 dq accumulator:
 // a fused kernel adds one float32 partial of every dq row per key tile into
 // global memory, and the L2's float32 reduction rate (a few TB/s) then bounds
 // the whole backward.  dq is also bitwise deterministic this way.
+// s2_bwd_dkdv_half_kernel (option S2_OPT_DKDV_HALF) is the dK/dV pass over
+// half query tiles with double-buffered score regions.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
