@@ -133,6 +133,31 @@ def test_scheduler_under_document_masks_visits_exactly_the_oracle_pairs(harness,
                     np.testing.assert_array_equal(vis.astype(bool), A, err_msg=where)
 
 
+@pytest.mark.parametrize("seed", range(24))
+def test_scheduler_under_random_document_layouts(harness, seed):
+    # random shape, valid length and document cuts (any position, any count) for all three traversals
+    r = np.random.default_rng(7000 + seed)
+    variant = int(r.integers(0, 3))
+    G = 256 * int(r.integers(1, 5))
+    N = G * int(r.integers(1, 3 if variant == 2 else 4))
+    if variant == 2:
+        G = N
+    nv = N if r.random() < 0.4 else int(r.integers(1, N + 1))
+    ids = np.zeros(N, dtype=np.int32)
+    for c in r.choice(np.arange(1, N), size=int(r.integers(0, 12)), replace=False):
+        ids[c:] += 1
+    bounds = np.ascontiguousarray(_bounds_of(ids))
+    same = ids[:, None] == ids[None, :]
+    for cls in ((0,) if variant == 2 else (0, 1)):
+        A = oracle.adjacency(N, G, nv, variant, cls) & same
+        for which in (0, 1, 2):
+            vis = np.zeros((N, N), dtype=np.uint8)
+            harness.s2h_visit_docs(N, G, nv, variant, cls, bounds.ctypes.data, which, vis.ctypes.data)
+            where = str((seed, N, G, nv, variant, cls, which))
+            assert vis.max() <= 1, "a pair was computed twice " + where
+            np.testing.assert_array_equal(vis.astype(bool), A, err_msg=where)
+
+
 def test_dq_traversal_without_documents(harness):
     for N, G, variant in ((1024, 512, 0), (1024, 512, 1), (768, 768, 2)):
         for nv in (N, N - 200):
