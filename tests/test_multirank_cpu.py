@@ -60,3 +60,34 @@ def test_two_rank_max_reduction_and_aggregate(tmp_path):
         assert r["clocks"]["sm_mhz"] == 1850.0       # median of the two ranks' medians
         # 2 ranks x 7e12 FLOPs over the slowest rank's 11 ms per step
         assert abs(r["value"] - 2 * 7.0e12 / 11e-3 / 1e12) < 1e-9
+
+
+def _bench(args, env_extra=None):
+    import subprocess
+
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, str(ROOT / "bench.py"), *args], capture_output=True, text=True,
+                          env=env, timeout=600, cwd=str(ROOT))
+
+
+def test_reference_arm_prints_the_contract_line():
+    # the reference arm times the float64 oracle on the host; no GPU involved
+    r = _bench(["--impl", "reference", "--steps", "2", "--warmup", "0", "--workload", "small_n1024_g256"])
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
+    assert d["steps"] == 2 and d["warmup"] >= 3 and d["higher_is_better"] is True
+    assert d["config"]["workload"] == "small_n1024_g256" and d["dtype"] == "f64"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_prints_nothing_on_other_ranks():
+    r = _bench(["--impl", "reference", "--steps", "1", "--workload", "small_n1024_g256"],
+               {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
