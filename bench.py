@@ -423,9 +423,12 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     s2.check_status()
     ms = start.elapsed_time(end)
-    per = {name: sum(e[a].elapsed_time(e[b]) for e in evs) / args.steps
-           for name, a, b in (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_dkdv", 2, 3), ("bwd_dq", 3, 4))
-           + ((("rope", 5, 0),) if args.rope else ())}
+    stages = (("fwd", 0, 1), ("bwd_prepare", 1, 2), ("bwd_dkdv", 2, 3), ("bwd_dq", 3, 4)) + (
+        (("rope", 5, 0),) if args.rope else ())
+    samples = {name: [e[a].elapsed_time(e[b]) for e in evs] for name, a, b in stages}
+    per = {name: sum(t) / args.steps for name, t in samples.items()}
+    # this rank's spread over the timed steps (the survey's protocol: median and minimum per pass)
+    per_spread = {name: {"median": statistics.median(t), "min": min(t)} for name, t in samples.items()}
     clocks = clk.summary()
 
     # e2e: the same step through the public API from pinned host buffers, copies included.
@@ -558,6 +561,7 @@ def run_ours(args, rank, world, local_rank):
                         "bf16_sustained": value / world / pk["bf16_sustained"],
                         "nominal_2250": value / world / 2250.0},
         "kernel_ms": per,
+        "kernel_ms_rank0_spread": per_spread,
         "useful_flops_per_step": flops_step,
         "exact_pair_tflops": (world * pairs * 14 * D / (ms_step * 1e-3) / 1e12) if pairs else None,
         "clocks": clocks,
@@ -569,6 +573,11 @@ def run_ours(args, rank, world, local_rank):
     line["config"]["backward"] = ("stored dS (dQ pass reads the dK/dV pass's dS tiles; workspace %.2f GB)"
                                   % (ws_bytes / 1e9) if stored else "recomputing dQ pass (workspace %.1f MB)"
                                   % (ws_bytes / 1e6))
+    if pairs and not args.doc_len:
+        # executed MMA work over the exact useful work: every visited 128 x 128 tile is
+        # multiplied in full, so the excess is the masked half of the diagonal tiles
+        tp = w.B * (w.H // 2) * (stored_tile_pairs(w, variant, 0) + stored_tile_pairs(w, variant, 1))
+        line["executed_over_useful"] = tp * 128 * 128 / pairs
     if stored and not args.doc_len:
         # the stored-dS dQ pass is HBM-bound: it reads one 32 KB dS tile per computed
         # tile pair, the K tiles and writes dq
