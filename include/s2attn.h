@@ -160,22 +160,6 @@ int s2attn_bwd_docs(const void* q, const void* k, const void* v, const void* o, 
                     int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant,
                     void* workspace, size_t workspace_bytes, int stages, void* stream);
 
-/* Process-wide options.  S2_OPT_FWD_PAIRS (value 0 or 1, default 0): run
- * the forward of D = 128 without documents on pairs of CTAs whose tensor-core
- * products span both (tcgen05 cta_group::2, M = 256 rows), halving the shared-
- * memory operand traffic per product; results equal the single-CTA forward
- * within rounding.  Slower than the default on the workloads measured so
- * far (2.97 against 2.25 ms on B1 H32 N32768 D128 G8192).  Not synchronised:
- * set it before launching work. */
-/* S2_OPT_DKDV_HALF (0 or 1, default 0): run the dK/dV pass over half query
- * tiles of 64 rows with its score regions double-buffered in tensor memory
- * (the products of the next half overlap the exponentials of the current
- * one); results equal the default pass within rounding.  Slower than the
- * default on the workloads measured so far (5.88 against 4.65 ms on
- * B1 H32 N32768 D128 G8192). */
-enum { S2_OPT_FWD_PAIRS = 1, S2_OPT_DKDV_HALF = 2 };
-int s2attn_set_option(int option, int value);
-
 /* Rotary position prologue ("4.1.2 · LongLoRA: 用S²-Attn完成长上下文微调" §1.1,
  * "RoPE使用原始位置"): Q and K are rotated at each token's ORIGINAL position
  * ID, never its index inside a group, with position interpolation p -> p·scale
@@ -286,15 +270,25 @@ int s2attn_graph_gap(const float* lse_s2, const float* lse_full, const void* o_s
  * owns the device heap, or a runtime held to a fixed memory footprint.  The
  * pages describe no such entry point; it exists for those callers only.
  * Instead of a caller-provided workspace it uses one file-scope device array
- * of S2_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until
- * the process exits.  Shapes whose s2attn_bwd_workspace_size() exceeds that
- * size are rejected with S2_ERR_UNSUPPORTED before anything is launched.
- * The first call on each device looks up the array's device address (with
- * that device current) and caches it, so make that first call before any
- * stream capture begins.  All calls share the one array: calls whose kernels
+ * of S2_NOALLOC_SCRATCH_BYTES.  Shapes whose s2attn_bwd_workspace_size()
+ * exceeds that size are rejected with S2_ERR_UNSUPPORTED before anything is
+ * launched.
+ * When the array is reserved: the driver reserves it when it loads the
+ * array's device module into a context, which under CUDA's default lazy
+ * module loading happens inside the FIRST call on each device (under
+ * CUDA_MODULE_LOADING=EAGER, when the context is created); it stays reserved
+ * until that context is destroyed.  A caller whose framework will claim the
+ * device heap should make one call at start-up, before the framework
+ * reserves its memory and outside any stream capture.  If the device has no
+ * room for the array at that first call, the call returns S2_ERR_CUDA with
+ * the driver's out-of-memory message and launches nothing.
+ * The first call on each device, with that device current, looks up the
+ * array's device address and caches it with the identity of the current
+ * context; a call in a later context of the device (after cudaDeviceReset)
+ * looks it up again.  All calls share the one array: calls whose kernels
  * overlap on the GPU (other streams, other host threads) race on it.  No
- * allocating routine is called; every call rewrites the statistics it reads
- * before reading them. */
+ * allocating routine is called by the library itself; every call rewrites
+ * the statistics it reads before reading them. */
 int s2attn_bwd_noalloc_v(const void* q, const void* k, const void* v, const void* o,
                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
                          int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid,
@@ -326,7 +320,7 @@ int s2attn_debug_wait_probe(int64_t budget_cycles, void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 108. */
+/* ABI version of this header (major*100 + minor): 200. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

@@ -50,7 +50,6 @@ SIGNATURES = {
     "s2attn_sp_halo_unpack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
-    "s2attn_set_option": ([_int, _int], _int),
     "s2attn_debug_wait_probe": ([_i64, _vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
     "s2attn_version": ([], _int),
@@ -201,23 +200,6 @@ def rope(q, k, positions=None, base: float = 10000.0, scale: float = 1.0, inplac
 
 
 S2_SP_KV, S2_SP_GRAD = 0, 1
-S2_OPT_FWD_PAIRS, S2_OPT_DKDV_HALF = 1, 2
-
-
-def s2attn_set_option(option, value) -> int:
-    return lib().s2attn_set_option(option, value)
-
-
-def set_dkdv_half(enabled: bool) -> None:
-    """Run the dK/dV pass over half query tiles (see include/s2attn.h)."""
-    _check(s2attn_set_option(S2_OPT_DKDV_HALF, 1 if enabled else 0))
-
-
-def set_fwd_pairs(enabled: bool) -> None:
-    """Run the D = 128 forward on CTA pairs (see include/s2attn.h)."""
-    _check(s2attn_set_option(S2_OPT_FWD_PAIRS, 1 if enabled else 0))
-
-
 def s2attn_sp_fwd(q, k, v, o, lse, B, L, H, D, G, n_valid, variant, rank, world, stream=None) -> int:
     return lib().s2attn_sp_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, L, H, D, G, n_valid, variant, rank,
                                world, _stream(stream))

@@ -13,7 +13,7 @@ PKG = Path(__file__).resolve().parent
 ROOT = PKG.parent
 CSRC = PKG / "csrc"
 LIB = PKG / "libs2attn.so"
-SOURCES = ["s2attn_api.cu", "s2_fwd.cu", "s2_fwd2.cu", "s2_bwd.cu", "s2_adj.cu", "s2_docs.cu", "s2_gap.cu", "s2_rope.cu", "s2_sp.cu", "s2attn_noalloc.cu"]
+SOURCES = ["s2attn_api.cu", "s2_fwd.cu", "s2_bwd.cu", "s2_adj.cu", "s2_docs.cu", "s2_gap.cu", "s2_rope.cu", "s2_sp.cu", "s2attn_noalloc.cu"]
 HEADERS = ["s2_index.cuh", "sm100_ptx.cuh", "s2_kernels.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

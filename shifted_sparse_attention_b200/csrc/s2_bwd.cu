@@ -30,8 +30,6 @@
 // a fused kernel adds one float32 partial of every dq row per key tile into
 // global memory, and the L2's float32 reduction rate (a few TB/s) then bounds
 // the whole backward.  dq is also bitwise deterministic this way.
-// s2_bwd_dkdv_half_kernel (option S2_OPT_DKDV_HALF) is the dK/dV pass over
-// half query tiles with double-buffered score regions.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -985,390 +983,11 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #undef sKt
 }
 
-// ------------------------------------------------------------------ dK, dV pass over half query tiles
-// The same pass as s2_bwd_dkdv_kernel with query tiles split in halves of 64
-// rows and the score regions double-buffered in TMEM: S^T and dP^T of half h
-// go to buffer h % 2 (64 columns each), so the products of half h + 1 are
-// already computed while the elementwise warpgroup h % 2 works on half h, and
-// the tensor core never waits for one half's exponentials behind its own
-// products.  TMEM (512 columns): S^T/P^T [64b, 64b + 64), dP^T/dS^T
-// [128 + 64b, ...), dV [256, 256 + D), dK [256 + D, 256 + 2D).  Warpgroup x
-// (warps 4x .. 4x + 3, thread = key row) handles the halves h = x (mod 2), all
-// 64 of their query columns.  Issue order per half h (one thread of warp 9):
-//     dV += P^T(h) dO(h),  dK += dS^T(h) Q(h),  S^T(h+2),  dP^T(h+2)
-// Q and dO halves stream through rings of four 16 KB slots.
-namespace dkdvh {
-
-constexpr int kHalf = 64;
-constexpr int kQSlots = 4, kOSlots = 4;
-enum Bar {
-  KV_FULL = 0,
-  Q_FULL = 1,     // + slot (4)
-  Q_EMPTY = 5,    // + slot (4)
-  O_FULL = 9,     // + slot (4)
-  O_EMPTY = 13,   // + slot (4): dV's commit + the 128 threads of the warpgroup after their dS step
-  S_FULL = 17,    // + buffer (2)
-  DP_FULL = 19,   // + buffer (2)
-  P_READY = 21,   // + buffer (2)
-  DS_READY = 23,  // + buffer (2)
-  ACC_DONE = 25,
-  NUM_BARS = 26
-};
-
-template <int D>
-struct Layout {
-  static constexpr int kTileBytes = kTile * D * 2;   // K or V tile
-  static constexpr int kHalfBytes = kHalf * D * 2;   // Q or dO half tile
-  static constexpr int kHalfChunk = kHalf * 64 * 2;  // 64 rows x 64 columns
-  static constexpr int kRowBytes = kHalf * 4;        // one float32 statistic of a half tile
-  static constexpr int kK = 0;
-  static constexpr int kV = kTileBytes;
-  static constexpr int kQ = 2 * kTileBytes;                  // + slot * kHalfBytes
-  static constexpr int kdO = kQ + kQSlots * kHalfBytes;      // + slot * kHalfBytes
-  static constexpr int kLse = kdO + kOSlots * kHalfBytes;    // -lse2 rows, + slot * kRowBytes
-  static constexpr int kDelta = kLse + kQSlots * kRowBytes;  // -Delta rows, + slot * kRowBytes
-  static constexpr int kBars = kDelta + kOSlots * kRowBytes;
-  static constexpr int kBytes = kBars + NUM_BARS * 8 + 16;
-};
-
-// The walk over half tiles: (query tile, half) after (qt, hf), or qt = -1.
-__device__ __forceinline__ void next_half(const Plan& p, const Unit& u, int lo, int hi, int& qt, int& hf) {
-  if (hf == 0) {
-    hf = 1;
-  } else {
-    qt = bwd::next_q(p, u, qt, lo, hi);
-    hf = 0;
-  }
-}
-
-}  // namespace dkdvh
-
-template <int D, bool kStoreDS>
-__global__ void __launch_bounds__(bwd::kThreads, 1)
-    s2_bwd_dkdv_half_kernel(const __grid_constant__ CUtensorMap tmQ64, const __grid_constant__ CUtensorMap tmK,
-                            const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO64,
-                            const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
-                            const __grid_constant__ Plan p, const float* __restrict__ delta,
-                            const float* __restrict__ lse2, __nv_bfloat16* __restrict__ ds_store,
-                            int* __restrict__ status) {
-  using namespace bwd;
-  using namespace dkdvh;
-  using L = dkdvh::Layout<D>;
-  constexpr int kChunks = D / 64;
-
-  Unit u;
-  if (!decode_kv_unit(p, blockIdx.x, u)) return;
-  extern __shared__ __align__(1024) uint8_t smem_kvh[];
-  if (smem_u32(smem_kvh) & 1023u) {
-    if (threadIdx.x == 0) atomicOr(status, 256);
-    return;
-  }
-  const int kt = u.t[0];
-  const int k0 = tile_orig(p, u, kt);
-  int lK, hK;
-  doc_span(p, u.b, k0, lK, hK);
-  const int q_first = !u.part[0] ? -1 : qtile_valid(p, u, kt) ? kt : next_q(p, u, kt, lK, hK);
-  const bool kvalid = q_first >= 0;
-
-  uint8_t* smem = smem_kvh;
-  const uint32_t sb = smem_u32(smem);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kBars + NUM_BARS * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const uint32_t sbar = sb + L::kBars;
-#define bar(i) (sbar + 8u * (uint32_t)(i))
-#define sQh(st) (sb + L::kQ + (uint32_t)(st) * L::kHalfBytes)
-#define sdOh(st) (sb + L::kdO + (uint32_t)(st) * L::kHalfBytes)
-  const uint32_t sK = sb + L::kK, sV = sb + L::kV;
-
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  if (threadIdx.x == 0) {
-    mbar_init(bar(KV_FULL), 1);
-    for (int i = 0; i < kQSlots; ++i) {
-      mbar_init(bar(Q_FULL + i), 1);
-      mbar_init(bar(Q_EMPTY + i), 1);
-    }
-    for (int i = 0; i < kOSlots; ++i) {
-      mbar_init(bar(O_FULL + i), 1);
-      mbar_init(bar(O_EMPTY + i), 1 + 128);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(S_FULL + b), 1);
-      mbar_init(bar(DP_FULL + b), 1);
-      mbar_init(bar(P_READY + b), 128);
-      mbar_init(bar(DS_READY + b), 128);
-    }
-    mbar_init(bar(ACC_DONE), 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-    fence_proxy_async_smem();
-  }
-  if (warp == 9) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tdV = tmem + 256, tdK = tmem + 256 + D;
-  const int row_base = u.b * p.N;
-  const size_t stat_base = ((size_t)u.b * p.H + u.h) * p.N;
-
-  if (warp == 8) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && kvalid) {
-      prefetch_tmap(&tmQ64);
-      prefetch_tmap(&tmdO64);
-      mbar_arrive_expect_tx(bar(KV_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < kChunks; ++c) {
-        tma_load_3d(sK + c * kChunkBytes, &tmK, c * 64, u.h, row_base + k0, bar(KV_FULL));
-        tma_load_3d(sV + c * kChunkBytes, &tmV, c * 64, u.h, row_base + k0, bar(KV_FULL));
-      }
-      int n = 0;
-      bool ok = true;
-      for (int qt = q_first, hf = 0; ok && qt >= 0; next_half(p, u, lK, hK, qt, hf), ++n) {
-        const int q0 = tile_orig(p, u, qt) + kHalf * hf;
-        const int sq = n % kQSlots, so = n % kOSlots;
-        if (n >= kQSlots) ok = s2_wait(bar(Q_EMPTY + sq), ((n / kQSlots) - 1) & 1, abort_flag, status, 8);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(Q_FULL + sq), L::kHalfBytes + L::kRowBytes);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(sQh(sq) + c * L::kHalfChunk, &tmQ64, c * 64, u.h, row_base + q0, bar(Q_FULL + sq));
-        bulk_load(sb + L::kLse + sq * L::kRowBytes, lse2 + stat_base + q0, L::kRowBytes, bar(Q_FULL + sq));
-        if (n >= kOSlots) ok = s2_wait(bar(O_EMPTY + so), ((n / kOSlots) - 1) & 1, abort_flag, status, 8);
-        if (!ok) break;
-        mbar_arrive_expect_tx(bar(O_FULL + so), L::kHalfBytes + L::kRowBytes);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(sdOh(so) + c * L::kHalfChunk, &tmdO64, c * 64, u.h, row_base + q0, bar(O_FULL + so));
-        bulk_load(sb + L::kDelta + so * L::kRowBytes, delta + stat_base + q0, L::kRowBytes, bar(O_FULL + so));
-      }
-      // the last loads must land before the CTA retires
-      for (int d = (n > kQSlots ? n - kQSlots : 0); d < n; ++d)
-        s2_wait(bar(Q_FULL + d % kQSlots), (d / kQSlots) & 1, abort_flag, status, 8);
-      for (int d = (n > kOSlots ? n - kOSlots : 0); d < n; ++d)
-        s2_wait(bar(O_FULL + d % kOSlots), (d / kOSlots) & 1, abort_flag, status, 8);
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && kvalid) {
-      constexpr uint32_t id_s = umma_idesc_bf16(128, kHalf, 0, 0);  // S^T, dP^T: M keys, N 64 queries
-      constexpr uint32_t id_acc = umma_idesc_bf16(128, D, 0, 1);    // dV, dK: A from TMEM, B MN-major
-      const uint64_t dK_km = umma_desc_sw128(sK, 16, 1024), dV_km = umma_desc_sw128(sV, 16, 1024);
-      const uint64_t dQ_km = umma_desc_sw128(sQh(0), 16, 1024), ddO_km = umma_desc_sw128(sdOh(0), 16, 1024);
-      const uint64_t dQ_mn = umma_desc_sw128(sQh(0), L::kHalfChunk, 1024);
-      const uint64_t ddO_mn = umma_desc_sw128(sdOh(0), L::kHalfChunk, 1024);
-      constexpr uint64_t kSlotStep = (uint64_t)(L::kHalfBytes >> 4);
-      // K-major B over a half tile: 32 bytes per K step inside a 64-row chunk, then a chunk
-#define S2_KMH_OFF(kk) ((uint64_t)((((kk) / 4) * L::kHalfChunk + ((kk) % 4) * 32) >> 4))
-      bool ok = s2_wait(bar(KV_FULL), 0, abort_flag, status, 16);
-      auto issue_s = [&](int h) {  // S^T(h) -> buffer h % 2, dP^T(h) -> buffer h % 2
-        const int sq = h % kQSlots, so = h % kOSlots, b = h % 2;
-        ok = ok && s2_wait(bar(Q_FULL + sq), (h / kQSlots) & 1, abort_flag, status, 16);
-        if (!ok) return;
-        tc_fence_after();
-        const uint64_t oq = (uint64_t)sq * kSlotStep, od = (uint64_t)so * kSlotStep;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + 64 * b, dK_km + S2_KM_OFF(kk), dQ_km + oq + S2_KMH_OFF(kk), id_s, kk > 0);
-        umma_commit(bar(S_FULL + b));
-        ok = s2_wait(bar(O_FULL + so), (h / kOSlots) & 1, abort_flag, status, 16);
-        if (!ok) return;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + 128 + 64 * b, dV_km + S2_KM_OFF(kk), ddO_km + od + S2_KMH_OFF(kk), id_s, kk > 0);
-        umma_commit(bar(DP_FULL + b));
-      };
-      // the walk, two halves ahead of the products that consume them
-      int qa = q_first, ha = 0;  // half h
-      int qb = qa, hb = ha;      // half h + 2
-      int nh = 0;                // halves issued (scores)
-      if (ok) {
-        issue_s(0);
-        ++nh;
-        next_half(p, u, lK, hK, qb, hb);
-        if (qb >= 0) {
-          issue_s(1);
-          ++nh;
-          next_half(p, u, lK, hK, qb, hb);
-        }
-      }
-      for (int h = 0; ok && qa >= 0; ++h) {
-        const int b = h % 2, sq = h % kQSlots, so = h % kOSlots;
-        const uint64_t oq = (uint64_t)sq * kSlotStep, od = (uint64_t)so * kSlotStep;
-        // dV += P^T(h) dO(h): K = 64 queries, 16 per step, P^T pairs at S + 8·kk
-        ok = s2_wait(bar(P_READY + b), (h / 2) & 1, abort_flag, status, 16);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kHalf / 16; ++kk)
-          umma_ts(tdV, tmem + 64 * b + 8 * kk, ddO_mn + od + S2_MN_OFF(kk), id_acc, (h > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(O_EMPTY + so));  // dV is the last MMA reading dO(h)
-        // dK += dS^T(h) Q(h)
-        ok = s2_wait(bar(DS_READY + b), (h / 2) & 1, abort_flag, status, 16);
-        if (!ok) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < kHalf / 16; ++kk)
-          umma_ts(tdK, tmem + 128 + 64 * b + 8 * kk, dQ_mn + oq + S2_MN_OFF(kk), id_acc,
-                  (h > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(Q_EMPTY + sq));
-        // scores of half h + 2 into the buffer just released (behind dV(h), dK(h))
-        if (qb >= 0) {
-          issue_s(nh);
-          ++nh;
-          next_half(p, u, lK, hK, qb, hb);
-        }
-        next_half(p, u, lK, hK, qa, ha);
-      }
-#undef S2_KMH_OFF
-      // every issued MMA must be complete before TMEM is read or released
-      umma_commit(bar(ACC_DONE));
-      s2_wait(bar(ACC_DONE), 0, abort_flag, status, 16);
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ elementwise warpgroups
-    const int x = warp / 4;                // halves h = x (mod 2)
-    const int j = (warp % 4) * 32 + lane;  // key row == TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
-    bool ok = true;
-    int n = 0;  // halves seen (both warpgroups walk all of them)
-    if (kvalid) {
-      const bool key_tile_ragged = k0 + kTile > p.n_valid;
-      const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
-      const uint32_t tS = tmem + lane_off + 64 * x, tdP = tmem + lane_off + 128 + 64 * x;
-      for (int qt = q_first, hf = 0; ok && qt >= 0; next_half(p, u, lK, hK, qt, hf), ++n) {
-        if ((n & 1) != x) continue;
-        const int sq = n % kQSlots, so = n % kOSlots, k = n / 2;  // k: this warpgroup's k-th half
-        // visible query columns of this half from key row j
-        const bool masked = (qt == kt) || key_tile_ragged || p.docs != nullptr;
-        int lo = 0, hi = kHalf;
-        if (masked) {
-          int a, bq;
-          key_cols(p, u, kt, qt, j, a, bq);
-          lo = a - kHalf * hf;
-          hi = bq - kHalf * hf;
-          lo = lo < 0 ? 0 : lo;
-          hi = hi > kHalf ? kHalf : hi;
-        }
-        // stored dS: row j of tile (qt, kt), query blocks [8hf, 8hf + 8)
-        uint4* ds_tile = nullptr;
-        if constexpr (kStoreDS)
-          ds_tile = reinterpret_cast<uint4*>(ds_store + ds_slot(p, u, qt, kt) * (kTile * kTile)) + (j >> 3) * 128 +
-                    (j & 7);
-        // P(h) = 2^(S·log2(e)/sqrt(D) - lse·log2(e)) -> P^T pairs over S columns [0, 32)
-        ok = s2_wait(bar(Q_FULL + sq), (n / kQSlots) & 1, abort_flag, status, 32);
-        if (ok) ok = s2_wait(bar(S_FULL + x), k & 1, abort_flag, status, 32);
-        if (!ok) break;
-        tc_fence_after();
-        const float2* nl = reinterpret_cast<const float2*>(smem + L::kLse + sq * L::kRowBytes);
-        uint32_t sv[64];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_wait_ld();
-        uint32_t pk[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 a = __ffma2_rn(make_float2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), c2, nl[i]);
-          float p0 = ex2(a.x), p1 = ex2(a.y);
-          if (masked) {
-            p0 = (2 * i >= lo && 2 * i < hi) ? p0 : 0.f;
-            p1 = (2 * i + 1 >= lo && 2 * i + 1 < hi) ? p1 : 0.f;
-          }
-          pk[i] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tS, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-        tmem_st16(tS + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(P_READY + x));
-        // dS(h) = P (dP - Delta) -> dS^T pairs over dP columns [0, 32)
-        ok = s2_wait(bar(O_FULL + so), (n / kOSlots) & 1, abort_flag, status, 32);
-        if (ok) ok = s2_wait(bar(DP_FULL + x), k & 1, abort_flag, status, 32);
-        if (!ok) break;
-        tc_fence_after();
-        const float2* nd = reinterpret_cast<const float2*>(smem + L::kDelta + so * L::kRowBytes);
-        uint32_t dp[64];
-        tmem_ld32(tdP, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tdP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
-        tmem_wait_ld();
-        uint32_t keep[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 d2 = __fadd2_rn(make_float2(__uint_as_float(dp[2 * i]), __uint_as_float(dp[2 * i + 1])), nd[i]);
-          const float2 pv = make_float2(__uint_as_float(pk[i] << 16), __uint_as_float(pk[i] & 0xffff0000u));
-          const float2 ds = __fmul2_rn(pv, d2);
-          keep[i] = pack_bf16(ds.x, ds.y);
-        }
-        tmem_st16(tdP, *reinterpret_cast<const uint32_t(*)[16]>(&keep[0]));
-        tmem_st16(tdP + 16, *reinterpret_cast<const uint32_t(*)[16]>(&keep[16]));
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(DS_READY + x));
-        mbar_arrive(bar(O_EMPTY + so));  // done with the -Delta rows of dO slot so
-        if constexpr (kStoreDS) {
-#pragma unroll
-          for (int v4 = 0; v4 < 8; ++v4)
-            __stcs(ds_tile + (8 * hf + v4) * 8,
-                   make_uint4(keep[4 * v4], keep[4 * v4 + 1], keep[4 * v4 + 2], keep[4 * v4 + 3]));
-        }
-      }
-    }
-    // ---------------------------------------------------------- epilogue: dK, dV
-    bool have = kvalid && ok && n > 0;
-    if (have) {
-      have = s2_wait(bar(ACC_DONE), 0, abort_flag, status, 32);
-      tc_fence_after();
-    }
-    const bool key_valid = k0 + j < p.n_valid;
-    const float scale = p.scale_log2 * 0.69314718055994531f;  // 1/sqrt(D)
-    // staging: dV -> Q slots 0-1 (32 KB), dK -> Q slots 2-3 (every MMA reading them has completed)
-    acc_to_smem<D>(tdV, lane_off, x, j, have, key_valid, 1.f, sQh(0));
-    acc_to_smem<D>(tdK, lane_off, x, j, have, key_valid, scale, sQh(2));
-    fence_proxy_async_smem();
-    named_bar_sync(2, 256);
-    if (threadIdx.x == 0) {
-      for (int c = 0; c < kChunks; ++c) {
-        tma_store_3d(&tmdV, sQh(0) + c * kChunkBytes, c * 64, u.h, row_base + k0);
-        tma_store_3d(&tmdK, sQh(2) + c * kChunkBytes, c * 64, u.h, row_base + k0);
-      }
-      tma_store_commit();
-      tma_store_wait_all();
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-#undef bar
-#undef sQh
-#undef sdOh
-}
-
 #undef S2_KM_OFF
 #undef S2_MN_OFF
 
 template <int D, bool kStoreDS>
-int launch_dkdv_half(const BwdArgs& a, int grid) {
-  constexpr int kBytes = dkdvh::Layout<D>::kBytes;
-  static_assert(kBytes <= 232448, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(s2_bwd_dkdv_half_kernel<D, kStoreDS>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);
-  if (e != cudaSuccess) return (int)e;
-  s2_bwd_dkdv_half_kernel<D, kStoreDS><<<grid, bwd::kThreads, kBytes, a.stream>>>(
-      *a.tmQ64, *a.tmK, *a.tmV, *a.tmdO64, *a.tmdK, *a.tmdV, a.plan, a.delta, a.lse2,
-      static_cast<__nv_bfloat16*>(a.ds), a.status);
-  return (int)cudaGetLastError();
-}
-
-template <int D, bool kStoreDS>
 int launch_dkdv(const BwdArgs& a, int grid) {
-  if (a.tmQ64) return launch_dkdv_half<D, kStoreDS>(a, grid);
   constexpr int kBytes = dkdv::Layout<D>::kBytes;
   cudaError_t e =
       cudaFuncSetAttribute(s2_bwd_dkdv_kernel<D, kStoreDS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kBytes);

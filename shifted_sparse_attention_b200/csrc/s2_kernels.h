@@ -15,7 +15,6 @@ struct FwdArgs {
   const CUtensorMap* tmK;
   const CUtensorMap* tmV;
   const CUtensorMap* tmO;
-  const CUtensorMap* tmK64;  // k in boxes of 64 rows (CTA-pair forward), or null
   Plan plan;
   float* lse;
   int* status;
@@ -37,20 +36,19 @@ struct BwdArgs {
   float* delta;       // workspace [B, H, N]: -(dout_i·o_i)
   float* lse2;        // workspace [B, H, N]: -lse_i·log2(e), -inf on padded rows
   void* ds;           // stored-dS workspace (bf16 tiles of 32 KB, see s2_index.cuh), or null
-  const CUtensorMap* tmQ64;   // q in boxes of 64 rows: the dK/dV pass over half query tiles, or null
-  const CUtensorMap* tmdO64;  // dout in boxes of 64 rows (with tmQ64)
   int* status;
   cudaStream_t stream;
 };
 
 int launch_fwd(const FwdArgs& a);
-// CTA-pair forward (D = 128, no documents); needs a.tmK64 (boxes of 64 rows of k).
-int launch_fwd_pair(const FwdArgs& a);
 // stages: 1 = prepare (Delta, lse2), 2 = dK/dV pass, 4 = dQ pass; with 8 the
 // dK/dV pass also stores dS and the dQ pass reads it instead of recomputing.
 int launch_bwd(const BwdArgs& a, int stages);
 // Sets the calling thread's s2attn_last_error() message; returns `code`.
 int report_error(int code, const char* fmt, ...);
+// Process-unique ID of the calling thread's current CUDA context (0 if unknown):
+// per-device caches of device addresses are valid only inside that context.
+unsigned long long current_context_id();
 
 int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
 // Failure-detection probe: a bounded wait on a barrier nothing completes.

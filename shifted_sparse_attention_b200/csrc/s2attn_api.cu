@@ -42,6 +42,7 @@ struct DeviceState {
   bool ready = false;
   bool supported = false;
   int* status = nullptr;
+  unsigned long long ctx_id = 0;  // context `status` belongs to
   EncodeTiledFn encode = nullptr;
   std::string why;
 };
@@ -60,8 +61,12 @@ int device_state(DeviceState** out) {
   // autograd worker threads may not have touched the runtime yet).
   e = cudaSetDevice(dev);
   if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaSetDevice: %s", cudaGetErrorString(e));
+  const unsigned long long ctx = s2::current_context_id();
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState& st = g_dev[dev];
+  // a new context of the device (e.g. after cudaDeviceReset) reloads the module:
+  // the status word's address must be looked up again
+  if (st.ready && st.supported && ctx != 0 && st.ctx_id != ctx) st.ready = false;
   if (!st.ready) {
     cudaDeviceProp prop;
     e = cudaGetDeviceProperties(&prop, dev);
@@ -75,6 +80,7 @@ int device_state(DeviceState** out) {
       e = cudaGetSymbolAddress(&sym, g_s2_status);
       if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
       st.status = static_cast<int*>(sym);
+      st.ctx_id = ctx;
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
       e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
@@ -91,11 +97,6 @@ int device_state(DeviceState** out) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-// S2_OPT_FWD_PAIRS: forward over CTA pairs where it applies (process-wide).
-int g_fwd_pairs = 0;
-// S2_OPT_DKDV_HALF: the dK/dV pass over half query tiles (process-wide).
-int g_dkdv_half = 0;
 
 // Shape rules of the method plus the kernels' own support limits.
 int validate(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant) {
@@ -142,6 +143,32 @@ int launch_status(int rc, const char* what) {
 }  // namespace
 
 namespace s2 {
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
 // Records a message for s2attn_last_error() from other translation units.
 int report_error(int code, const char* fmt, ...) {
   char buf[512];
@@ -156,19 +183,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 108; }
-
-int s2attn_set_option(int option, int value) {
-  if (option == S2_OPT_FWD_PAIRS) {
-    g_fwd_pairs = value != 0;
-    return S2_OK;
-  }
-  if (option == S2_OPT_DKDV_HALF) {
-    g_dkdv_half = value != 0;
-    return S2_OK;
-  }
-  return fail(S2_ERR_INVALID_ARG, "unknown option %d", option);
-}
+int s2attn_version(void) { return 200; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -188,17 +203,10 @@ static int fwd_launch(const void* q, const void* k, const void* v, void* o, floa
     return rc;
   s2::FwdArgs a;
   a.tmQ = &tq; a.tmK = &tk; a.tmV = &tv; a.tmO = &to;
-  a.tmK64 = nullptr;
   a.plan = plan;
   a.lse = lse;
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
-  if (g_fwd_pairs && D == 128 && plan.docs == nullptr) {
-    CUtensorMap tk64;
-    if ((rc = make_tmap(st, &tk64, k, B, N, H, D, 64))) return rc;
-    a.tmK64 = &tk64;
-    return launch_status(s2::launch_fwd_pair(a), "forward (CTA pairs)");
-  }
   return launch_status(s2::launch_fwd(a), "forward");
 }
 
@@ -337,15 +345,6 @@ static int bwd_launch(const void* q, const void* k, const void* v, const void* o
   a.lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + sb);
   // stored dS: bf16 tiles of 32 KB after the row statistics (bulk copies need 16-byte alignment)
   a.ds = stored ? static_cast<char*>(workspace) + stats : nullptr;
-  a.tmQ64 = nullptr;
-  a.tmdO64 = nullptr;
-  CUtensorMap tq64, tdo64;
-  if (g_dkdv_half) {
-    if ((rc = make_tmap(st, &tq64, q, B, N, H, D, 64)) || (rc = make_tmap(st, &tdo64, dout, B, N, H, D, 64)))
-      return rc;
-    a.tmQ64 = &tq64;
-    a.tmdO64 = &tdo64;
-  }
   a.status = st->status;
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_status(s2::launch_bwd(a, stages), "backward");

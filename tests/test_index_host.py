@@ -198,7 +198,7 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 108
+    assert L.s2attn_version() == 200
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
@@ -398,3 +398,18 @@ def test_bench_tile_pair_count_matches_the_kernels_traversal(harness):
         if variant == 2:
             counted *= 2  # both heads of the dense graph are class 0
         assert int(w.sum()) == counted, (N, G, nv, variant, int(w.sum()), counted)
+
+
+def test_bench_pair_count_matches_the_oracle():
+    # bench.py prices exact-pair throughput (and the executed-over-useful ratio) on a
+    # closed count of visible pairs per head class, padding included
+    import bench
+    from types import SimpleNamespace
+
+    import oracle
+
+    for (N, G, nv, variant) in [(1024, 256, 1024, 0), (1024, 256, 1000, 0), (2048, 512, 1283, 1),
+                                (2048, 512, 300, 1), (1024, 1024, 900, 2), (4096, 1024, 4096, 1)]:
+        c0, c1 = bench.pair_counts(SimpleNamespace(N=N, G=G, valid=nv), variant)
+        assert c0 == oracle.pair_count(N, G, nv, variant, 0), (N, G, nv, variant)
+        assert c1 == oracle.pair_count(N, G, nv, variant, 0 if variant == 2 else 1), (N, G, nv, variant)

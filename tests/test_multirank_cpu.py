@@ -83,6 +83,7 @@ def test_reference_arm_prints_the_contract_line():
     assert d["config"]["workload"] == "small_n1024_g256" and d["dtype"] == "f64"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["cpu_baseline"]["value"] == d["value"]
+    assert set(d["cpu_baseline"]["seconds"]) == {"fwd", "bwd", "total"} and d["cpu_baseline"]["cpu_model"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 

@@ -395,3 +395,44 @@ def test_planted_mistakes_are_caught():
         assert not _pins_pass(pred), name
     # and the real predicate passes the same check
     assert _pins_pass(lambda N, G, i, j: oracle.visible(N, G, N, STRICT, 1, i, j))
+
+
+# --------------------------------------------------------------------------
+# segment identities of the gradients (used by the full-size GPU checks)
+
+
+@pytest.mark.parametrize("variant,n_valid", [(STRICT, None), (ROLLED, None), (DENSE, None), (STRICT, 45),
+                                             (ROLLED, 51), (DENSE, 37)])
+def test_gradient_segment_identities(variant, n_valid):
+    """Each softmax row sums to one, so dV summed over a segment's keys equals dO
+    summed over its valid queries; sum_j dS_ij = g_i·o_i - Delta_i = 0, so dK sums to
+    zero over a segment ([PT] §3's gradient).  A dropped Delta term or a
+    mis-normalised softmax breaks one of them.  The segment layout the GPU tests use
+    (tests/seg_layout.py) is checked here against the oracle's own matrices: every
+    row of a segment sees only keys of that segment, and its last row sees all of
+    them."""
+    from tests.seg_layout import segments
+
+    B, N, H, D, G = 1, 64, 4, 8, 16
+    nv = N if n_valid is None else n_valid
+    x = synthetic.draw(B, N, H, D, seed=12)
+    res = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, n_valid=nv)
+    g = _f64(x["dout"])[0].numpy().copy()
+    g[nv:] = 0
+    for h in range(H):
+        cls = 0 if variant == DENSE else int(h >= H // 2)
+        A = oracle.adjacency(N, G, nv, variant, cls)
+        segs = segments(N, G, variant, cls)
+        covered = np.zeros(N, dtype=int)
+        for seg in segs:
+            rows = np.concatenate([np.arange(a, b) for a, b in seg])
+            covered[rows] += 1
+            outside = np.ones(N, dtype=bool)
+            outside[rows] = False
+            assert not A[np.ix_(rows, np.nonzero(outside)[0])].any(), (h, seg)
+            last = rows[rows < nv][-1] if (rows < nv).any() else None
+            if last is not None:
+                assert A[last, rows[rows < nv]].all(), (h, seg)
+            np.testing.assert_allclose(res["dv"][0, rows, h].sum(0), g[rows, h].sum(0), atol=1e-11, rtol=0)
+            np.testing.assert_allclose(res["dk"][0, rows, h].sum(0), 0.0, atol=1e-11, rtol=0)
+        assert (covered == 1).all()
