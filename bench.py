@@ -49,6 +49,9 @@ def parse():
                     help="pack documents of this many tokens (document mask); reports exact-pair TFLOP/s")
     ap.add_argument("--sp-emulate", type=int, default=0, metavar="W",
                     help="sequence parallelism: run W ranks' shards (halo exchange + rank kernels) in turn on this GPU")
+    ap.add_argument("--sp", action="store_true",
+                    help="sequence parallelism over the torchrun ranks: each GPU holds a G-aligned shard of the "
+                         "sequence and exchanges the half-group halo over NCCL (strong scaling)")
     ap.add_argument("--recompute-dq", action="store_true",
                     help="dQ pass recomputes S and dP (8 MB workspace) instead of reading the stored dS")
     ap.add_argument("--rope", action="store_true",
@@ -741,6 +744,126 @@ def run_ours(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def sp_layout(N, G, n_valid, world):
+    """Shard length and each rank's valid rows when a sequence of N (padded) rows,
+    n_valid of them valid, is cut into `world` G-aligned shards: rank r holds
+    original positions [rL, rL + L).  Padding may sit only on the last rank
+    (the rank kernels' rule), so every other rank must be full."""
+    if world < 1 or N % (world * G):
+        raise ValueError("N=%d is not a multiple of world x G = %d x %d" % (N, world, G))
+    L = N // world
+    valid = [max(0, min(L, n_valid - r * L)) for r in range(world)]
+    if any(v != L for v in valid[:-1]) or valid[-1] < 1:
+        raise ValueError("the padding of n_valid=%d does not fall on the last of %d shards of %d rows" % (
+            n_valid, world, L))
+    return L, valid
+
+
+def run_sp(args, rank, world, local_rank):
+    """Sequence parallelism over the torchrun ranks ("4.1.2 · LongLoRA:
+    用S²-Attn完成长上下文微调" §1.1, Sequence Parallel通信).  Each rank holds the
+    G-aligned shard [rL, rL + L) of the workload in extended buffers (halo
+    rows first).  One step per rank: the K/V halo exchange (pack, NCCL
+    send/receive with both neighbours, unpack), the rank's forward and its
+    stored-dS backward, and the halo rows' gradients back to their owner.
+    value = the whole sequence's useful FLOPs / the slowest rank's step time
+    (strong scaling: the total work is fixed as ranks are added)."""
+    import torch
+    import torch.distributed as dist
+
+    from shifted_sparse_attention_b200 import binding as s2
+    from shifted_sparse_attention_b200 import sp
+    from shifted_sparse_attention_b200 import synthetic
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synthetic.WORKLOADS[args.workload]
+    variant = w.variants[0] if args.variant is None else args.variant
+    if variant not in (0, 1):
+        raise SystemExit("--sp runs the strict and rolled variants")
+    B, N, H, D, G = w.B, w.N, w.H, w.D, w.G
+    L, valid = sp_layout(N, G, w.valid, world)
+    s = G // 2
+    nv = valid[rank]
+    x = synthetic.draw(B, N, H, D, seed=w.seed, sharpen_k=w.sharpen_k)
+    t = {}
+    for name in ("q", "k", "v", "dout"):
+        e = sp.extended(B, L, H, D, G, dev)
+        e.zero_()
+        sp.shard(e, G).copy_(x[name][:, rank * L:(rank + 1) * L])
+        t[name] = e
+    del x
+    attn = sp.SequenceParallelS2Attn(G, variant)
+    o = torch.empty_like(t["q"])
+    lse = torch.empty((B, H, s + L), dtype=torch.float32, device=dev)
+    grads = tuple(torch.empty_like(t["q"]) for _ in range(3))
+    ws_bytes = s2.s2attn_sp_ds_workspace_size(B, L, H, D, G, variant, rank, world)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        attn.exchange_kv(t["k"], t["v"])
+        if ev is not None:
+            ev[1].record(stream)
+        attn.forward(t["q"], t["k"], t["v"], n_valid=nv, out=o, lse=lse, exchange=False)
+        if ev is not None:
+            ev[2].record(stream)
+        attn.backward(t["q"], t["k"], t["v"], o, t["dout"], lse, n_valid=nv, grads=grads, workspace=ws,
+                      exchange=False, stored_ds=True)
+        if ev is not None:
+            ev[3].record(stream)
+        attn.exchange_grad(grads[1], grads[2])
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    s2.check_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(*_gpu_ids(local_rank)) as clk:
+        time.sleep(0.2)
+        for i in range(args.steps):
+            step(evs[i])
+        torch.cuda.synchronize()
+    dist.barrier()
+    s2.check_status()
+    ms = sum(e[0].elapsed_time(e[4]) for e in evs)
+    parts = (("halo_kv", 0, 1), ("fwd", 1, 2), ("bwd", 2, 3), ("halo_grad", 3, 4))
+    per = {name: sum(e[a].elapsed_time(e[b]) for e in evs) / args.steps for name, a, b in parts}
+    ms, per, clocks = combine_ranks(ms, per, clk.summary(), dev)
+    if rank != 0:
+        return
+    pk = peaks()
+    ms_step = ms / args.steps
+    flops = w.formula_flops(passes="fwd+bwd")
+    value = flops / (ms_step * 1e-3) / 1e12
+    to0, frm0 = sp.peers(0, world, variant)
+    line = {
+        "metric": METRIC + " (sequence parallel over %d GPUs)" % world,
+        "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": dict(_config(w, variant), parallelism="sp%d" % world, shard_rows=L,
+                       backward="stored dS", halo="NCCL point-to-point, %d bytes per direction"
+                       % s2.s2attn_sp_halo_bytes(B, H, D, G)),
+        "pct_of_peak": {"bf16_burst": value / world / pk["bf16_burst"],
+                        "bf16_sustained": value / world / pk["bf16_sustained"]},
+        "stage_ms_max_over_ranks": per,
+        "clocks": clocks,
+        # per step and rank: halo pack/unpack kernels where the rank sends/receives,
+        # the forward, the backward's three stages
+        "gpu_launches": args.steps * sum(
+            4 + (2 if sp.peers(r, world, variant)[0] is not None else 0)
+            + (2 if sp.peers(r, world, variant)[1] is not None else 0) for r in range(world)),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_sp_emulated(args):
     """Sequence-parallel step of W ranks, run one rank after another on this GPU.
 
@@ -869,19 +992,27 @@ def main():
             raise SystemExit("--sp-emulate runs on one GPU")
         run_sp_emulated(args)
         return
-    if world > 1:
+    if world > 1 or args.sp:
         import datetime
 
         import torch
         import torch.distributed as dist
 
         torch.cuda.set_device(local_rank)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        if world == 1:  # --sp on one GPU: a process group of one rank
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", "29531")
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.sp:
+            run_sp(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
+        if world > 1 or args.sp:
             import torch.distributed as dist
 
             dist.destroy_process_group()

@@ -92,3 +92,19 @@ def test_reference_arm_prints_nothing_on_other_ranks():
                {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_sp_layout_cuts_g_aligned_shards_with_padding_on_the_last():
+    # bench.py --sp: rank r holds [rL, rL + L); only the last rank may hold padding
+    import bench
+
+    assert bench.sp_layout(32768, 8192, 32768, 1) == (32768, [32768])
+    assert bench.sp_layout(32768, 8192, 32768, 4) == (8192, [8192] * 4)
+    assert bench.sp_layout(106496, 8192, 100000, 13) == (8192, [8192] * 12 + [100000 - 12 * 8192])
+    assert bench.sp_layout(12288, 1536, 12288, 8) == (1536, [1536] * 8)
+    import pytest
+
+    with pytest.raises(ValueError):
+        bench.sp_layout(32768, 8192, 32768, 8)  # shards of 4096 < G
+    with pytest.raises(ValueError):
+        bench.sp_layout(4096, 1024, 2000, 4)  # padding on ranks 1..3
