@@ -294,11 +294,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         bulk_load(sb + L::kDelta + so * L::kRowBytes, delta + stat_base + q0, L::kRowBytes, bar(O_FULL + so));
         ++n;
       }
-      // the last loads must land before the CTA retires
+      // the last loads must land before the CTA retires (also after an abort)
+      s2_wait_drain(bar(KV_FULL), 0, status, 8);
       for (int d = (n > kQSlots ? n - kQSlots : 0); d < n; ++d)
-        s2_wait(bar(Q_FULL + d % kQSlots), (d / kQSlots) & 1, abort_flag, status, 8);
+        s2_wait_drain(bar(Q_FULL + d % kQSlots), (d / kQSlots) & 1, status, 8);
       for (int d = (n > kOSlots ? n - kOSlots : 0); d < n; ++d)
-        s2_wait(bar(O_FULL + d % kOSlots), (d / kOSlots) & 1, abort_flag, status, 8);
+        s2_wait_drain(bar(O_FULL + d % kOSlots), (d / kOSlots) & 1, status, 8);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -371,9 +372,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         qt = qn;
         qn = qnn;
       }
-      // every issued MMA must be complete before TMEM is read or released
+      // every issued MMA must be complete before TMEM is read or released (also after an abort)
       umma_commit(bar(ACC_DONE));
-      s2_wait(bar(ACC_DONE), 0, abort_flag, status, 16);
+      s2_wait_drain(bar(ACC_DONE), 0, status, 16);
     }
     __syncwarp();
   } else {
@@ -655,12 +656,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         kb = kc;
         kc = kc >= 0 ? next_k(p, u, kc, lQ, hQ) : -1;
       }
-      // the last loads must land before the CTA retires
+      // the last loads must land before the CTA retires (also after an abort)
       for (int d = (eK > kKSlots ? eK - kKSlots : 0); d < eK; ++d)
-        s2_wait(bar(K_FULL + d % kKSlots), (d / kKSlots) & 1, abort_flag, status, 1);
+        s2_wait_drain(bar(K_FULL + d % kKSlots), (d / kKSlots) & 1, status, 1);
       for (int d = (eV > kVSlots ? eV - kVSlots : 0); d < eV; ++d)
-        s2_wait(bar(V_FULL + d % kVSlots), (d / kVSlots) & 1, abort_flag, status, 1);
-      s2_wait(bar(Q_FULL), 0, abort_flag, status, 1);
+        s2_wait_drain(bar(V_FULL + d % kVSlots), (d / kVSlots) & 1, status, 1);
+      s2_wait_drain(bar(Q_FULL), 0, status, 1);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -722,9 +723,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (jj + 1 < T) issue_dp(jj + 1);  // dP(jj) was read before DS_READY(jj)
         if (jj + 2 < T) issue_s(jj + 2);   // behind dQ(jj), the last reader of this S buffer
       }
-      // every issued MMA must be complete before TMEM is read or released
+      // every issued MMA must be complete before TMEM is read or released (also after an abort)
       umma_commit(bar(DQ_DONE));
-      s2_wait(bar(DQ_DONE), 0, abort_flag, status, 2);
+      s2_wait_drain(bar(DQ_DONE), 0, status, 2);
     }
     __syncwarp();
   } else {
@@ -916,9 +917,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         const int row = row_base + tile_orig(p, u, k);
         for (int c = 0; c < kChunks; ++c) tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
       }
-      // the last loads must land before the CTA retires
+      // the last loads must land before the CTA retires (also after an abort)
       for (int d = (e > kStages ? e - kStages : 0); d < e; ++d)
-        s2_wait(bar(FULL + d % kStages), (d / kStages) & 1, abort_flag, status, 1);
+        s2_wait_drain(bar(FULL + d % kStages), (d / kStages) & 1, status, 1);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -944,9 +945,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
                   (jj > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(EMPTY + st));
       }
-      // every issued MMA must be complete before TMEM is read or released
+      // every issued MMA must be complete before TMEM is read or released (also after an abort)
       umma_commit(bar(DQ_DONE));
-      s2_wait(bar(DQ_DONE), 0, abort_flag, status, 2);
+      s2_wait_drain(bar(DQ_DONE), 0, status, 2);
     }
     __syncwarp();
   } else {

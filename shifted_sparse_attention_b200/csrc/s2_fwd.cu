@@ -193,9 +193,10 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (kn >= 0) load(&tmK, kn);
         kc = kn;
       }
-      // drain: the last loads must land before the CTA retires
+      // drain: the last loads must land before the CTA retires (also after an abort)
       for (int d = (e > kSlots ? e - kSlots : 0); d < e; ++d)
-        s2_wait(bar(KV_FULL + d % kSlots), (d / kSlots) & 1, abort_flag, status, 1);
+        s2_wait_drain(bar(KV_FULL + d % kSlots), (d / kSlots) & 1, status, 1);
+      s2_wait_drain(bar(Q_FULL), 0, status, 1);
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -286,9 +287,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         eV = eV2;
         eK = eK2;
       }
-      // every issued MMA must be complete before TMEM is released
+      // every issued MMA must be complete before TMEM is released (also after an abort)
       umma_commit(bar(MMA_DONE));
-      s2_wait(bar(MMA_DONE), 0, abort_flag, status, 2);
+      s2_wait_drain(bar(MMA_DONE), 0, status, 2);
     }
     __syncwarp();
   } else if (warp < 8) {

@@ -7,7 +7,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
@@ -34,12 +33,6 @@ int fail(int code, const char* fmt, ...) {
 // Timeout / abort status word written by the kernels (bit flags per role).
 __device__ int g_s2_status;
 
-// Work-ticket counters of the persistent kernels: zero at module load, left at
-// zero by every launch that completes.  Launches take them round-robin, so up
-// to kTicketSlots launches can be in flight on one device without sharing one.
-constexpr int kTicketSlots = 4096;
-__device__ unsigned int g_s2_tickets[kTicketSlots];
-
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -49,9 +42,6 @@ struct DeviceState {
   bool ready = false;
   bool supported = false;
   int* status = nullptr;
-  unsigned int* tickets = nullptr;  // g_s2_tickets
-  std::atomic<unsigned int> next_ticket{0};
-  int num_sms = 0;
   unsigned long long ctx_id = 0;  // context `status` belongs to
   EncodeTiledFn encode = nullptr;
   std::string why;
@@ -91,10 +81,6 @@ int device_state(DeviceState** out) {
       if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
       st.status = static_cast<int*>(sym);
       st.ctx_id = ctx;
-      e = cudaGetSymbolAddress(&sym, g_s2_tickets);
-      if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-      st.tickets = static_cast<unsigned int*>(sym);
-      st.num_sms = prop.multiProcessorCount;
       cudaDriverEntryPointQueryResult q;
       void* fn = nullptr;
       e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
@@ -112,10 +98,6 @@ int device_state(DeviceState** out) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// This launch's work-ticket counter.
-unsigned int* ticket_counter(DeviceState* st) {
-  return st->tickets + st->next_ticket.fetch_add(1u, std::memory_order_relaxed) % kTicketSlots;
-}
 
 // Shape rules of the method plus the kernels' own support limits.
 int validate(int64_t B, int64_t N, int64_t H, int64_t D, int64_t G, int64_t n_valid, int variant) {

@@ -78,26 +78,6 @@ __device__ __forceinline__ bool s2_wait_drain(uint32_t bar, uint32_t parity, int
   return true;
 }
 
-// ---------------------------------------------------------------- persistent scheduling
-// Work tickets of a persistent launch: every CTA takes tickets from a counter
-// in global memory until one is past `total`.  Each CTA takes exactly one
-// such ticket, so the CTA holding the last of them (total + ctas - 1) is the
-// last to touch the counter, and resets it for the next launch on the stream.
-// claim_ticket issues the atomic; its result is needed only by settle_ticket,
-// so a CTA can claim its next ticket early and let the round trip to L2
-// (about 2 us under load) overlap its current work.
-__device__ __forceinline__ unsigned int claim_ticket(unsigned int* counter) { return atomicAdd(counter, 1u); }
-__device__ __forceinline__ int settle_ticket(unsigned int* counter, unsigned int t, int total) {
-  if ((int)t >= total) {
-    if ((int)t == total + (int)gridDim.x - 1) atomicExch(counter, 0u);
-    return -1;
-  }
-  return (int)t;
-}
-__device__ __forceinline__ int take_ticket(unsigned int* counter, int total) {
-  return settle_ticket(counter, claim_ticket(counter), total);
-}
-
 // ---------------------------------------------------------------- proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
