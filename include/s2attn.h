@@ -67,7 +67,8 @@ enum {
   S2_ERR_SHAPE = -2,       /* H, G, N, n_valid violate the divisibility / range rules */
   S2_ERR_UNSUPPORTED = -3, /* valid for the method but not for these kernels (D, G/2 % 128, GPU) */
   S2_ERR_CUDA = -4,        /* a CUDA runtime call failed */
-  S2_ERR_TIMEOUT = -5      /* a kernel gave up waiting on a barrier */
+  S2_ERR_TIMEOUT = -5,     /* a kernel gave up waiting on a barrier */
+  S2_ERR_BOUNDS = -6       /* the debug build found an index outside its bounds (see below) */
 };
 
 /* Forward.  Writes o [B,N,H,D] (bf16) and lse [B,H,N] (fp32) for all N rows. */
@@ -305,9 +306,39 @@ int s2attn_bwd_noalloc_v(const void* q, const void* k, const void* v, const void
 int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
                            int format, void* out, void* stream);
 
-/* Synchronizes `stream` and reports (then clears) a kernel timeout recorded
- * on the current device since the last check: S2_OK or S2_ERR_TIMEOUT. */
+/* Synchronizes `stream` and reports (then clears) a kernel timeout, or a
+ * bounds violation of the debug build, recorded on the current device since
+ * the last check: S2_OK, S2_ERR_TIMEOUT or S2_ERR_BOUNDS (the latter first). */
 int s2attn_check_status(void* stream);
+
+/* Bounds-checked build.  The library can also be built as
+ * libs2attn_debug.so (the same sources with -DS2_DEBUG_BOUNDS): there, before
+ * every access, each kernel checks the tile origins it computes against [0, N)
+ * and against the rows that may hold them (query tiles [q_begin, n_valid),
+ * key tiles [k_begin, n_valid) of the plan), its TMA row coordinates against
+ * the tensor, the global indices it stores to, the stored-dS slots against the
+ * workspace, and the TMEM columns it addresses against the 512 allocated.
+ * The first violation on the device is recorded (site, value, bounds); the
+ * access is skipped and the kernel gives up as on a timeout, without a trap,
+ * so the context stays usable.  Results of the debug build equal the normal
+ * build's bit for bit.
+ * s2attn_debug_bounds_checked: 1 in the debug build, 0 in the normal one.
+ * s2attn_debug_bounds_report: synchronizes `stream` and writes the first
+ * recorded violation as out[4] = {site, value, lower bound (inclusive), upper
+ * bound (exclusive)}, or zeros if there is none; it does not clear the record
+ * (s2attn_check_status does).  Sites: 1-4 forward (Q tile, K/V tile, output
+ * row or lse index, TMEM), 5-9 dK/dV pass (K/V tile, Q/dO tile or statistics
+ * rows, stored-dS slot, output row, TMEM), 10-13 dQ passes (Q/dO tile or
+ * statistics, K/V tile or stored-dS slot, output row, TMEM), 14 the probe
+ * below.
+ * s2attn_debug_bounds_probe: launches one thread that runs the same check on
+ * `value` against [lo, hi) with site 14 and touches no memory on its result,
+ * so the recording path can be exercised without a real violation.  In the
+ * normal build the check is compiled out and nothing is recorded.  Returns
+ * S2_ERR_INVALID_ARG if lo > hi. */
+int s2attn_debug_bounds_checked(void);
+int s2attn_debug_bounds_report(int64_t* out, void* stream);
+int s2attn_debug_bounds_probe(int64_t value, int64_t lo, int64_t hi, void* stream);
 
 /* Failure-detection probe: launches one CTA whose wait on a barrier that
  * nothing completes runs out after `budget_cycles` SM clocks (in [1000, 4e9]);
@@ -320,7 +351,7 @@ int s2attn_debug_wait_probe(int64_t budget_cycles, void* stream);
 /* Message for the last non-OK status returned to the calling thread. */
 const char* s2attn_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 200. */
+/* ABI version of this header (major*100 + minor): 201. */
 int s2attn_version(void);
 
 #ifdef __cplusplus

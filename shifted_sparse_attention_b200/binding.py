@@ -7,6 +7,7 @@ sm_100a part, calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 from pathlib import Path
 
@@ -14,8 +15,11 @@ import torch
 
 STRICT, ROLLED, DENSE_CAUSAL = 0, 1, 2
 S2_OK, S2_ERR_INVALID_ARG, S2_ERR_SHAPE, S2_ERR_UNSUPPORTED, S2_ERR_CUDA, S2_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+S2_ERR_BOUNDS = -6
 
 LIB_PATH = Path(__file__).resolve().parent / "libs2attn.so"
+# the same library with the kernels' bounds checks compiled in (include/s2attn.h)
+DEBUG_LIB_PATH = Path(__file__).resolve().parent / "libs2attn_debug.so"
 
 # name -> (argtypes, restype), mirroring include/s2attn.h
 _i64, _int, _vp, _fp, _sz = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
@@ -50,6 +54,9 @@ SIGNATURES = {
     "s2attn_sp_halo_unpack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
+    "s2attn_debug_bounds_checked": ([], _int),
+    "s2attn_debug_bounds_report": ([_vp, _vp], _int),
+    "s2attn_debug_bounds_probe": ([_i64, _i64, _i64, _vp], _int),
     "s2attn_debug_wait_probe": ([_i64, _vp], _int),
     "s2attn_last_error": ([], ctypes.c_char_p),
     "s2attn_version": ([], _int),
@@ -64,19 +71,49 @@ class S2AttnError(RuntimeError):
         self.code = code
 
 
+def _load(path: Path) -> ctypes.CDLL:
+    if not path.exists():
+        raise ImportError("%s is not built; run `python -m shifted_sparse_attention_b200.build`" % path.name)
+    L = ctypes.CDLL(str(path))
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    return L
+
+
 def lib() -> ctypes.CDLL:
     """Load libs2attn.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not LIB_PATH.exists():
-            raise ImportError("libs2attn.so is not built; run `python -m shifted_sparse_attention_b200.build`")
-        L = ctypes.CDLL(str(LIB_PATH))
-        for name, (args, res) in SIGNATURES.items():
-            fn = getattr(L, name)
-            fn.argtypes = args
-            fn.restype = res
-        _lib = L
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+_debug_lib = None
+
+
+@contextlib.contextmanager
+def debug_library():
+    """Route every call of this module through libs2attn_debug.so (the kernels
+    with their bounds checks) inside the block."""
+    global _lib, _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(DEBUG_LIB_PATH)
+    saved = lib()
+    _lib = _debug_lib
+    try:
+        yield _debug_lib
+    finally:
+        _lib = saved
+
+
+def bounds_report(stream=None) -> tuple:
+    """(site, value, lower, upper) of the first bounds violation the debug build
+    recorded on this device, or zeros (include/s2attn.h)."""
+    out = (ctypes.c_int64 * 4)()
+    _check(lib().s2attn_debug_bounds_report(ctypes.cast(out, ctypes.c_void_p), _stream(stream)))
+    return tuple(int(v) for v in out)
 
 
 def _check(rc: int) -> None:
@@ -347,6 +384,10 @@ def debug_adjacency(N: int, G: int, variant: int, head_class: int, n_valid: int 
         out = torch.empty((N, 4), dtype=torch.int32, device=device)
     _check(s2attn_debug_adjacency(N, G, nv, variant, head_class, fmt, out))
     return out
+
+
+def s2attn_debug_bounds_probe(value, lo, hi, stream=None) -> int:
+    return lib().s2attn_debug_bounds_probe(value, lo, hi, _stream(stream))
 
 
 def s2attn_debug_wait_probe(budget_cycles, stream=None) -> int:

@@ -9,6 +9,7 @@
 // scheduler and the masks independently of any floating-point result.
 #include <cuda_runtime.h>
 
+#include "s2_debug.cuh"
 #include "s2_index.cuh"
 #include "s2_kernels.h"
 #include "sm100_ptx.cuh"
@@ -106,6 +107,18 @@ __global__ void s2_wait_probe_kernel(int* __restrict__ status, long long budget)
 
 int launch_wait_probe(int* status, long long budget, cudaStream_t stream) {
   s2_wait_probe_kernel<<<1, 64, 0, stream>>>(status, budget);
+  return (int)cudaGetLastError();
+}
+
+// One thread runs the kernels' bounds check on a value the caller chose.  No
+// memory access depends on the outcome: this exercises the recording path
+// (first violation wins, later ones only set the flag) without any fault.
+__global__ void s2_bounds_probe_kernel(int* __restrict__ status, long long v, long long lo, long long hi) {
+  (void)S2_IN(kSiteProbe, v, lo, hi);
+}
+
+int launch_bounds_probe(int* status, long long v, long long lo, long long hi, cudaStream_t stream) {
+  s2_bounds_probe_kernel<<<1, 1, 0, stream>>>(status, v, lo, hi);
   return (int)cudaGetLastError();
 }
 

@@ -34,6 +34,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "s2_debug.cuh"
 #include "s2_index.cuh"
 #include "s2_kernels.h"
 #include "sm100_ptx.cuh"
@@ -271,15 +272,26 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmdO);
       mbar_arrive_expect_tx(bar(KV_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < kChunks; ++c) {
-        tma_load_3d(sK + c * kChunkBytes, &tmK, c * 64, u.h, row_base + k0, bar(KV_FULL));
-        tma_load_3d(sV + c * kChunkBytes, &tmV, c * 64, u.h, row_base + k0, bar(KV_FULL));
+      if (S2_IN(kSiteKvK, k0, p.k_begin, p.n_valid) && S2_IN(kSiteKvK, k0, 0, p.N - kTile + 1) &&
+          S2_IN(kSiteKvK, row_base + k0, 0, (long long)p.B * p.N - kTile + 1)) {
+        for (int c = 0; c < kChunks; ++c) {
+          tma_load_3d(sK + c * kChunkBytes, &tmK, c * 64, u.h, row_base + k0, bar(KV_FULL));
+          tma_load_3d(sV + c * kChunkBytes, &tmV, c * 64, u.h, row_base + k0, bar(KV_FULL));
+        }
+      } else {
+        *abort_flag = 1;  // the debug build skips the access and gives up
       }
       int n = 0;
       bool ok = true;
       for (int qt = q_first; ok && qt >= 0; qt = next_q(p, u, qt, lK, hK)) {
         const int q0 = tile_orig(p, u, qt);
         const int sq = n % kQSlots, so = n % kOSlots;
+        if (!(S2_IN(kSiteKvQ, q0, p.q_begin, p.n_valid) && S2_IN(kSiteKvQ, q0, 0, p.N - kTile + 1) &&
+              S2_IN(kSiteKvQ, row_base + q0, 0, (long long)p.B * p.N - kTile + 1) &&
+              S2_IN(kSiteKvQ, stat_base + q0, 0, (long long)p.B * p.H * p.N - kTile + 1))) {
+          *abort_flag = 1;
+          break;
+        }
         if (n >= kQSlots) ok = s2_wait(bar(Q_EMPTY + sq), ((n / kQSlots) - 1) & 1, abort_flag, status, 8);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(Q_FULL + sq), L::kTileBytes + L::kRowBytes);
@@ -384,6 +396,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
     bool ok = true;
     int n = 0;
+    // R1, R2, dV, dK within the 512 allocated columns
+    if (!S2_IN(kSiteKvTmem, 256 + 2 * D, 257, 513)) *abort_flag = 1;
     if (kvalid) {
       const bool key_tile_ragged = k0 + kTile > p.n_valid;
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
@@ -436,9 +450,15 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         // [8b, 8b + 8) sits at (j / 8)·2048 + b·128 + (j % 8)·16 bytes, so one block
         // of a warp's 32 rows is four 128-byte runs
         uint4* ds_tile = nullptr;
-        if constexpr (kStoreDS)
-          ds_tile = reinterpret_cast<uint4*>(ds_store + ds_slot(p, u, qt, kt) * (kTile * kTile)) + (j >> 3) * 128 +
-                    (j & 7);
+        if constexpr (kStoreDS) {
+          const long long slot = ds_slot(p, u, qt, kt);
+          if (!S2_IN(kSiteKvDs, slot, 0, (long long)p.B * p.H * p.ds_head_tiles)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          ds_tile = reinterpret_cast<uint4*>(ds_store + slot * (kTile * kTile)) + (j >> 3) * 128 + (j & 7);
+        }
         // dS(n) = P (dP - Delta) -> dS^T pairs into R2
         ok = s2_wait(bar(O_FULL + sd), (n / kOSlots) & 1, abort_flag, status, 32);
         if (ok) ok = s2_wait(bar(DP_FULL), n & 1, abort_flag, status, 32);
@@ -491,7 +511,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     acc_to_smem<D>(tdK, lane_off, x, j, have, key_valid, scale, sQ(1));
     fence_proxy_async_smem();
     named_bar_sync(2, 256);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && S2_IN(kSiteKvOut, k0, 0, p.N - kTile + 1) &&
+        S2_IN(kSiteKvOut, row_base + k0, 0, (long long)p.B * p.N - kTile + 1)) {
       for (int c = 0; c < kChunks; ++c) {
         tma_store_3d(&tmdV, sQ(0) + c * kChunkBytes, c * 64, u.h, row_base + k0);
         tma_store_3d(&tmdK, sQ(1) + c * kChunkBytes, c * 64, u.h, row_base + k0);
@@ -623,9 +644,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(bar(Q_FULL), 2 * L::kTileBytes);
-      for (int c = 0; c < kChunks; ++c) {
-        tma_load_3d(sQ + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(Q_FULL));
-        tma_load_3d(sdO + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(Q_FULL));
+      if (S2_IN(kSiteDqQ, q0, p.q_begin, p.n_valid) && S2_IN(kSiteDqQ, q0, 0, p.N - kTile + 1) &&
+          S2_IN(kSiteDqQ, row_base + q0, 0, (long long)p.B * p.N - kTile + 1)) {
+        for (int c = 0; c < kChunks; ++c) {
+          tma_load_3d(sQ + c * kChunkBytes, &tmQ, c * 64, u.h, row_base + q0, bar(Q_FULL));
+          tma_load_3d(sdO + c * kChunkBytes, &tmdO, c * 64, u.h, row_base + q0, bar(Q_FULL));
+        }
+      } else {
+        *abort_flag = 1;
       }
       int eK = 0, eV = 0;
       bool ok = true;
@@ -638,8 +664,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) return;
         mbar_arrive_expect_tx(full, L::kTileBytes);
         const uint32_t dst = isK ? sKs(slot) : sVs(slot);
-        const int row = row_base + tile_orig(p, u, k);
-        for (int c = 0; c < kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, isK ? &tmK : &tmV, c * 64, u.h, row, full);
+        const int x0 = tile_orig(p, u, k);
+        const int row = row_base + x0;
+        if (S2_IN(kSiteDqK, x0, p.k_begin, p.n_valid) && S2_IN(kSiteDqK, x0, 0, p.N - kTile + 1) &&
+            S2_IN(kSiteDqK, row, 0, (long long)p.B * p.N - kTile + 1)) {
+          for (int c = 0; c < kChunks; ++c) tma_load_3d(dst + c * kChunkBytes, isK ? &tmK : &tmV, c * 64, u.h, row, full);
+        } else {
+          *abort_flag = 1;
+        }
         if (isK) ++eK; else ++eV;
       };
       // consumption order: K(0), K(1), V(0), then per j: V(j+1), K(j+2)
@@ -738,6 +770,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     int jj = 0;
     if (qvalid) {
       const size_t stat_at = ((size_t)u.b * p.H + u.h) * p.N + q0 + r;
+      // S0, S1, dP, dQ within the 512 allocated columns; the row's statistics
+      if (!(S2_IN(kSiteDqTmem, 384 + D, 385, 513) && S2_IN(kSiteDqQ, stat_at, 0, (long long)p.B * p.H * p.N)))
+        *abort_flag = 1;
       const float nl = lse2[stat_at], nd = delta[stat_at];  // -lse·log2(e) (-inf if padded), -Delta
       const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
       const float2 nl2 = make_float2(nl, nl), nd2 = make_float2(nd, nd);
@@ -803,7 +838,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     acc_to_smem<D>(tdQ, lane_off, x, r, have, row_valid, scale, sQ);
     fence_proxy_async_smem();
     named_bar_sync(2, 256);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && S2_IN(kSiteDqOut, q0, 0, p.N - kTile + 1) &&
+        S2_IN(kSiteDqOut, row_base + q0, 0, (long long)p.B * p.N - kTile + 1)) {
       for (int c = 0; c < kChunks; ++c) tma_store_3d(&tmdQ, sQ + c * kChunkBytes, c * 64, u.h, row_base + q0);
       tma_store_commit();
       tma_store_wait_all();
@@ -913,9 +949,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (e >= kStages) ok = s2_wait(bar(EMPTY + st), ((e / kStages) - 1) & 1, abort_flag, status, 1);
         if (!ok) break;
         mbar_arrive_expect_tx(bar(FULL + st), L::kStageBytes);
-        bulk_load(sDS(st), ds + ds_slot(p, u, qt, k) * (kTile * kTile), L::kDSBytes, bar(FULL + st));
-        const int row = row_base + tile_orig(p, u, k);
-        for (int c = 0; c < kChunks; ++c) tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
+        const long long slot = ds_slot(p, u, qt, k);
+        const int x0 = tile_orig(p, u, k);
+        const int row = row_base + x0;
+        if (S2_IN(kSiteDqK, slot, 0, (long long)p.B * p.H * p.ds_head_tiles) &&
+            S2_IN(kSiteDqK, x0, p.k_begin, p.n_valid) && S2_IN(kSiteDqK, x0, 0, p.N - kTile + 1) &&
+            S2_IN(kSiteDqK, row, 0, (long long)p.B * p.N - kTile + 1)) {
+          bulk_load(sDS(st), ds + slot * (kTile * kTile), L::kDSBytes, bar(FULL + st));
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(sKt(st) + c * kChunkBytes, &tmK, c * 64, u.h, row, bar(FULL + st));
+        } else {
+          *abort_flag = 1;
+        }
       }
       // the last loads must land before the CTA retires (also after an abort)
       for (int d = (e > kStages ? e - kStages : 0); d < e; ++d)
@@ -966,7 +1011,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     acc_to_smem<D>(tdQ, lane_off, x, r, have, row_valid, scale, sDS(0));
     fence_proxy_async_smem();
     named_bar_sync(2, 256);
-    if (threadIdx.x == 0) {
+    if (threadIdx.x == 0 && S2_IN(kSiteDqOut, q0, 0, p.N - kTile + 1) &&
+        S2_IN(kSiteDqOut, row_base + q0, 0, (long long)p.B * p.N - kTile + 1)) {
       for (int c = 0; c < kChunks; ++c) tma_store_3d(&tmdQ, sDS(0) + c * kChunkBytes, c * 64, u.h, row_base + q0);
       tma_store_commit();
       tma_store_wait_all();

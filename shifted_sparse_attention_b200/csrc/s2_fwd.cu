@@ -32,6 +32,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "s2_debug.cuh"
 #include "s2_index.cuh"
 #include "s2_kernels.h"
 #include "sm100_ptx.cuh"
@@ -167,7 +168,13 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
 #pragma unroll
       for (int x = 0; x < 2; ++x) {
         if (!(x ? pB : pA)) continue;
-        const int row = row_base + tile_orig(p, u, x ? tB : tA);
+        const int x0 = tile_orig(p, u, x ? tB : tA);
+        const int row = row_base + x0;
+        if (!(S2_IN(kSiteFwdQ, x0, p.q_begin, p.n_valid) && S2_IN(kSiteFwdQ, x0, 0, p.N - kTile + 1) &&
+              S2_IN(kSiteFwdQ, row, 0, (long long)p.B * p.N - kTile + 1))) {
+          *abort_flag = 1;  // the debug build skips the access and gives up
+          continue;
+        }
         for (int c = 0; c < kChunks; ++c)
           tma_load_3d(sQ(x) + c * kChunkBytes, &tmQ, c * 64, u.h, row, bar(Q_FULL));
       }
@@ -178,9 +185,15 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         if (e >= kSlots) ok = s2_wait(bar(KV_EMPTY + slot), ((e / kSlots) - 1) & 1, abort_flag, status, 1);
         if (!ok) return;
         mbar_arrive_expect_tx(bar(KV_FULL + slot), L::kKVBytes);
-        const int row = row_base + tile_orig(p, u, k);
-        for (int c = 0; c < kChunks; ++c)
-          tma_load_3d(sKV(slot) + c * kChunkBytes, tm, c * 64, u.h, row, bar(KV_FULL + slot));
+        const int x0 = tile_orig(p, u, k);
+        const int row = row_base + x0;
+        if (S2_IN(kSiteFwdKV, x0, p.k_begin, p.n_valid) && S2_IN(kSiteFwdKV, x0, 0, p.N - kTile + 1) &&
+            S2_IN(kSiteFwdKV, row, 0, (long long)p.B * p.N - kTile + 1)) {
+          for (int c = 0; c < kChunks; ++c)
+            tma_load_3d(sKV(slot) + c * kChunkBytes, tm, c * 64, u.h, row, bar(KV_FULL + slot));
+        } else {
+          *abort_flag = 1;
+        }
         ++e;
       };
       // consumption order: K(k0), then per key tile V(k), K(next k)
@@ -303,6 +316,9 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
     const int tx = x ? tB : tA;
     const bool px = x ? pB : pA;
     const int lx = x ? lB : lA, hx = x ? hB : hA;
+    // S_x and O_x within the 512 allocated columns
+    if (!(S2_IN(kSiteFwdTmem, x * 128 + 128, 1, 257) && S2_IN(kSiteFwdTmem, 256 + x * D + D, 257, 513)))
+      *abort_flag = 1;
     if (tx >= 0) {
       const int q0 = tile_orig(p, u, tx);
       const bool row_valid = (q0 + r) < p.n_valid;
@@ -423,10 +439,12 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
         }
       }
       const float lse_v = (have && row_valid) ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-      lse[((size_t)u.b * p.H + u.h) * p.N + q0 + r] = lse_v;
+      const size_t lse_at = ((size_t)u.b * p.H + u.h) * p.N + q0 + r;
+      if (S2_IN(kSiteFwdOut, lse_at, 0, (long long)p.B * p.H * p.N)) lse[lse_at] = lse_v;
+      const bool out_in = S2_IN(kSiteFwdOut, q0, 0, p.N - kTile + 1);
       fence_proxy_async_smem();
       named_bar_sync(1 + x, 128);
-      if (r == 0) {
+      if (r == 0 && out_in) {
         for (int c = 0; c < kChunks; ++c)
           tma_store_3d(&tmO, sQ(x) + c * kChunkBytes, c * 64, u.h, row_base + q0);
         tma_store_commit();

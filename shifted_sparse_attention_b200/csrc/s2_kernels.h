@@ -53,6 +53,7 @@ unsigned long long current_context_id();
 int launch_adjacency(const Plan& p, int head_class, int format, void* out, cudaStream_t stream);
 // Failure-detection probe: a bounded wait on a barrier nothing completes.
 int launch_wait_probe(int* status, long long budget, cudaStream_t stream);
+int launch_bounds_probe(int* status, long long v, long long lo, long long hi, cudaStream_t stream);
 
 // Training / inference graph gap: per-row rho and output shift, per (head
 // class, bucket) statistics float32 [2][kGapBuckets][4].

@@ -13,6 +13,7 @@
 #include <string>
 
 #include "../../include/s2attn.h"
+#include "s2_debug.cuh"
 #include "s2_index.cuh"
 #include "s2_kernels.h"
 
@@ -30,8 +31,10 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
-// Timeout / abort status word written by the kernels (bit flags per role).
-__device__ int g_s2_status;
+// Status area written by the kernels: [0] flag bits (timeouts per role, and
+// the debug build's bounds flag), then the debug build's first bounds
+// violation (s2_debug.cuh).
+__device__ int g_s2_status[s2::kStatusInts];
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -184,7 +187,7 @@ int report_error(int code, const char* fmt, ...) {
 
 extern "C" {
 
-int s2attn_version(void) { return 200; }
+int s2attn_version(void) { return 201; }
 
 const char* s2attn_last_error(void) { return g_last_error.c_str(); }
 
@@ -520,20 +523,59 @@ int s2attn_debug_wait_probe(int64_t budget_cycles, void* stream) {
                        "wait probe");
 }
 
-int s2attn_check_status(void* stream) {
+int s2attn_debug_bounds_probe(int64_t value, int64_t lo, int64_t hi, void* stream) {
+  if (lo > hi) return fail(S2_ERR_INVALID_ARG, "bounds probe: lower bound %lld above upper %lld", (long long)lo,
+                           (long long)hi);
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc) return rc;
+  return launch_status(s2::launch_bounds_probe(st->status, (long long)value, (long long)lo, (long long)hi,
+                                               static_cast<cudaStream_t>(stream)),
+                       "bounds probe");
+}
+
+// The status area after the stream's work (synchronises the stream).
+static int read_status(void* stream, int (&area)[s2::kStatusInts]) {
   DeviceState* st = nullptr;
   int rc = device_state(&st);
   if (rc) return rc;
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(S2_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
-  int flags = 0;
-  e = cudaMemcpyFromSymbol(&flags, g_s2_status, sizeof(int));
-  if (e != cudaSuccess) return fail(S2_ERR_CUDA, "reading the status word: %s", cudaGetErrorString(e));
-  if (flags) {
-    const int zero = 0;
-    cudaMemcpyToSymbol(g_s2_status, &zero, sizeof(int));
-    return fail(S2_ERR_TIMEOUT, "a kernel gave up waiting on a barrier (role flags 0x%x)", flags);
+  e = cudaMemcpy(area, st->status, sizeof area, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(S2_ERR_CUDA, "reading the status area: %s", cudaGetErrorString(e));
+  return S2_OK;
+}
+
+int s2attn_check_status(void* stream) {
+  int area[s2::kStatusInts];
+  int rc = read_status(stream, area);
+  if (rc) return rc;
+  const int flags = area[0];
+  if (!flags) return S2_OK;
+  DeviceState* st = nullptr;
+  device_state(&st);
+  const int zero[s2::kStatusInts] = {};
+  cudaMemcpy(st->status, zero, sizeof zero, cudaMemcpyHostToDevice);
+  if (flags & s2::kBoundsFlag) {
+    const long long* r = reinterpret_cast<const long long*>(area + 4);
+    return fail(S2_ERR_BOUNDS, "bounds check failed at site %d: value %lld outside [%lld, %lld) (flags 0x%x)",
+                area[2], r[0], r[1], r[2], flags);
   }
+  return fail(S2_ERR_TIMEOUT, "a kernel gave up waiting on a barrier (role flags 0x%x)", flags);
+}
+
+int s2attn_debug_bounds_checked(void) { return s2::kBoundsChecked ? 1 : 0; }
+
+int s2attn_debug_bounds_report(int64_t* out, void* stream) {
+  if (!out) return fail(S2_ERR_INVALID_ARG, "null output pointer");
+  int area[s2::kStatusInts];
+  int rc = read_status(stream, area);
+  if (rc) return rc;
+  const long long* r = reinterpret_cast<const long long*>(area + 4);
+  out[0] = area[1] ? area[2] : 0;
+  out[1] = area[1] ? r[0] : 0;
+  out[2] = area[1] ? r[1] : 0;
+  out[3] = area[1] ? r[2] : 0;
   return S2_OK;
 }
 

@@ -198,7 +198,27 @@ def test_library_exports_every_declared_symbol(abi):
     L = abi.lib()
     for name in declared:
         assert hasattr(L, name)
-    assert L.s2attn_version() == 200
+    assert L.s2attn_version() == 201
+    assert L.s2attn_debug_bounds_checked() == 0
+
+
+def test_debug_library_exports_the_same_symbols_with_checks_compiled_in(abi):
+    """libs2attn_debug.so is the same ABI; only the kernels carry the bounds checks."""
+    header = (ROOT / "include" / "s2attn.h").read_text()
+    declared = set(re.findall(r"\b(s2attn_\w+)\s*\(", header))
+    nm = subprocess.run(["nm", "-D", "--defined-only", str(abi.DEBUG_LIB_PATH)], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (s2attn_\w+)", nm))
+    assert declared <= exported, declared - exported
+    with abi.debug_library() as D:
+        assert D.s2attn_version() == 201
+        assert D.s2attn_debug_bounds_checked() == 1
+        assert abi.lib() is D
+    assert abi.lib().s2attn_debug_bounds_checked() == 0
+    # host validation is shared: a bad shape fails before any launch in both builds
+    fake = 1 << 20
+    with abi.debug_library() as D:
+        rc = D.s2attn_fwd_v(fake, fake, fake, fake, fake, 1, 1000, 8, 64, 256, 1000, 0, None)
+    assert rc == abi.S2_ERR_SHAPE
 
 
 def test_host_validation_rejects_bad_shapes_before_any_launch(abi):
