@@ -306,6 +306,14 @@ int s2attn_bwd_noalloc_v(const void* q, const void* k, const void* v, const void
 int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
                            int format, void* out, void* stream);
 
+/* Debug: the same dump under a document mask (packed sequences, see
+ * s2attn_doc_bounds): the pairs the document-aware kernels visit for one
+ * sequence.  doc_bounds is int32 [N, 2] of that sequence (device memory,
+ * 8-byte aligned), as s2attn_doc_bounds writes it for B = 1.  A row's
+ * visited keys are still at most two intervals in format 1. */
+int s2attn_debug_adjacency_docs(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                                const int32_t* doc_bounds, int format, void* out, void* stream);
+
 /* Synchronizes `stream` and reports (then clears) a kernel timeout, or a
  * bounds violation of the debug build, recorded on the current device since
  * the last check: S2_OK, S2_ERR_TIMEOUT or S2_ERR_BOUNDS (the latter first). */

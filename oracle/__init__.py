@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
         i32p = ctypes.POINTER(ctypes.c_int32)
         L.s2o_pair_count_docs.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int, i32p]
         L.s2o_pair_count_docs.restype = i64
+        L.s2o_adjacency_docs.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int, i32p, u8p]
+        L.s2o_adjacency_docs.restype = None
+        L.s2o_adjacency_row_docs.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int, i32p, i64, u8p]
+        L.s2o_adjacency_row_docs.restype = None
         L.s2o_attention.argtypes = [u16p, u16p, u16p, u16p, i32p, i64, i64, i64, i64, i64, i64,
                                     ctypes.c_int, i64, i64, i64p, i64, dp, dp, dp, dp, dp]
         L.s2o_attention.restype = ctypes.c_int
@@ -116,6 +120,25 @@ def pair_count_docs(N: int, G: int, n_valid: int, variant: int, head_class: int,
     d = np.ascontiguousarray(np.asarray(doc, dtype=np.int32))
     assert d.shape == (N,)
     return int(lib().s2o_pair_count_docs(N, G, n_valid, variant, head_class, _ptr(d, ctypes.c_int32)))
+
+
+def adjacency_docs(N: int, G: int, n_valid: int, variant: int, head_class: int, doc) -> np.ndarray:
+    """A^(head_class) restricted to same-document pairs (doc: N per-position IDs), [N, N] bool."""
+    d = np.ascontiguousarray(np.asarray(doc, dtype=np.int32))
+    assert d.shape == (N,)
+    out = np.zeros((N, N), dtype=np.uint8)
+    lib().s2o_adjacency_docs(N, G, n_valid, variant, head_class, _ptr(d, ctypes.c_int32), _ptr(out, ctypes.c_uint8))
+    return out.astype(bool)
+
+
+def adjacency_row_docs(N: int, G: int, n_valid: int, variant: int, head_class: int, doc, i: int) -> np.ndarray:
+    """Row i of adjacency_docs as a boolean vector of length N."""
+    d = np.ascontiguousarray(np.asarray(doc, dtype=np.int32))
+    assert d.shape == (N,)
+    out = np.zeros(N, dtype=np.uint8)
+    lib().s2o_adjacency_row_docs(N, G, n_valid, variant, head_class, _ptr(d, ctypes.c_int32), i,
+                                 _ptr(out, ctypes.c_uint8))
+    return out.astype(bool)
 
 
 def _docs(doc, B: int, N: int):

@@ -119,6 +119,22 @@ int64_t s2o_pair_count_docs(int64_t N, int64_t G, int64_t n_valid, int variant, 
   return c;
 }
 
+/* Explicit boolean matrix under a document mask (doc: [N] IDs of one batch
+ * row): out[i*N + j] = A^(c)[i][j] and doc[i] == doc[j]. */
+void s2o_adjacency_docs(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                        const int32_t* doc, uint8_t* out) {
+  for (int64_t i = 0; i < N; ++i)
+    for (int64_t j = 0; j < N; ++j)
+      out[i * N + j] = (uint8_t)(s2o_visible(N, G, n_valid, variant, head_class, i, j) && doc[i] == doc[j]);
+}
+
+/* One row of the document-masked matrix: out[j] = A^(c)[i][j] and doc[i] == doc[j]. */
+void s2o_adjacency_row_docs(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                            const int32_t* doc, int64_t i, uint8_t* out) {
+  for (int64_t j = 0; j < N; ++j)
+    out[j] = (uint8_t)(s2o_visible(N, G, n_valid, variant, head_class, i, j) && doc[i] == doc[j]);
+}
+
 /* bf16 bit pattern -> double (exact). */
 static double bf16_to_double(uint16_t b) {
   uint32_t u = ((uint32_t)b) << 16;

@@ -53,6 +53,7 @@ SIGNATURES = {
     "s2attn_sp_halo_pack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_sp_halo_unpack": ([_vp, _vp, _vp, _i64, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "s2attn_debug_adjacency": ([_i64, _i64, _i64, _int, _int, _int, _vp, _vp], _int),
+    "s2attn_debug_adjacency_docs": ([_i64, _i64, _i64, _int, _int, _vp, _int, _vp, _vp], _int),
     "s2attn_check_status": ([_vp], _int),
     "s2attn_debug_bounds_checked": ([], _int),
     "s2attn_debug_bounds_report": ([_vp, _vp], _int),
@@ -296,6 +297,11 @@ def s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, out, stream=
     return lib().s2attn_debug_adjacency(N, G, n_valid, variant, head_class, fmt, _ptr(out), _stream(stream))
 
 
+def s2attn_debug_adjacency_docs(N, G, n_valid, variant, head_class, doc_bounds, fmt, out, stream=None) -> int:
+    return lib().s2attn_debug_adjacency_docs(N, G, n_valid, variant, head_class, _ptr(doc_bounds), fmt, _ptr(out),
+                                             _stream(stream))
+
+
 def s2attn_check_status(stream=None) -> int:
     return lib().s2attn_check_status(_stream(stream))
 
@@ -375,14 +381,19 @@ def backward(q, k, v, o, dout, lse, G: int, variant: int = STRICT, n_valid: int 
 
 
 def debug_adjacency(N: int, G: int, variant: int, head_class: int, n_valid: int | None = None,
-                    fmt: int = 0, device="cuda"):
-    """Visited (query, key) pattern of one head class, from the kernels' scheduler."""
+                    fmt: int = 0, device="cuda", docs=None):
+    """Visited (query, key) pattern of one head class, from the kernels' scheduler.
+    docs: optional document bounds [1, N, 2] or [N, 2] (from doc_bounds) of one sequence."""
     nv = N if n_valid is None else int(n_valid)
     if fmt == 0:
         out = torch.empty((N, (N + 31) // 32), dtype=torch.int32, device=device)
     else:
         out = torch.empty((N, 4), dtype=torch.int32, device=device)
-    _check(s2attn_debug_adjacency(N, G, nv, variant, head_class, fmt, out))
+    if docs is None:
+        _check(s2attn_debug_adjacency(N, G, nv, variant, head_class, fmt, out))
+    else:
+        _check(s2attn_debug_adjacency_docs(N, G, nv, variant, head_class, _bounds(docs.reshape(1, N, 2), 1, N), fmt,
+                                           out))
     return out
 
 

@@ -17,7 +17,10 @@
 namespace s2 {
 
 // One CTA per work unit of a head of class `cls`; thread = one row of the
-// unit's two query tiles.
+// unit's two query tiles.  With a document mask (p.docs, one batch row) the
+// walk is the document-aware forward's: query tiles that hold a valid row,
+// key tiles that meet the span of the query tile's documents, and each row's
+// columns clipped to its document.
 __global__ void __launch_bounds__(256) s2_adjacency_kernel(const __grid_constant__ Plan p, int cls, int format,
                                                            uint32_t* __restrict__ bits,
                                                            int* __restrict__ intervals) {
@@ -32,11 +35,22 @@ __global__ void __launch_bounds__(256) s2_adjacency_kernel(const __grid_constant
     for (int w = 0; w < words; ++w) bits[(size_t)row * words + w] = 0u;
   int iv[4] = {-1, -1, -1, -1};
   int nint = 0;
+  // under a document mask: the forward's tile test (the span of the documents
+  // touching the query tile) and its per-row column range (row_cols)
+  int dlo = 0, dhi = p.N;
+  if (p.docs && u.part[x]) doc_span(p, u.b, tile_orig(p, u, u.t[x]), dlo, dhi);
   for (int k = 0; k <= u.t[x]; ++k) {
-    if (!tile_takes(p, u, x, k) || !ktile_valid(p, u, k)) continue;
-    const int lim = col_limit(p, u, u.t[x], k, r);
-    if (lim <= 0) continue;
-    const int lo = tile_orig(p, u, k), hi = lo + lim - 1;
+    if (!ktile_valid(p, u, k)) continue;
+    int c0 = 0, c1 = 0;
+    if (p.docs) {
+      if (!u.part[x] || !tile_meets(tile_orig(p, u, k), dlo, dhi)) continue;
+      row_cols(p, u, u.t[x], k, r, c0, c1);
+    } else {
+      if (!tile_takes(p, u, x, k)) continue;
+      c1 = col_limit(p, u, u.t[x], k, r);
+    }
+    if (c1 <= c0) continue;
+    const int lo = tile_orig(p, u, k) + c0, hi = tile_orig(p, u, k) + c1 - 1;
     if (format == 0) {
       for (int j = lo; j <= hi; ++j) bits[(size_t)row * words + j / 32] |= 1u << (j % 32);
     } else {

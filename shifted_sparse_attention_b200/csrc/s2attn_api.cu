@@ -496,8 +496,8 @@ int s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const
                       stream);
 }
 
-int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class, int format,
-                           void* out, void* stream) {
+static int adjacency_impl(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                          const int32_t* doc_bounds, int format, void* out, void* stream) {
   // D does not enter the pattern; validate with a supported D.
   int rc = validate(1, N, 2, 128, G, n_valid, variant);
   if (rc) return rc;
@@ -509,8 +509,21 @@ int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, i
   DeviceState* st = nullptr;
   if ((rc = device_state(&st))) return rc;
   s2::Plan p = s2::make_plan(1, (int)N, 2, 128, (int)G, (int)n_valid, variant);
+  p.docs = doc_bounds;
   const int cls = (variant == S2_DENSE_CAUSAL) ? 0 : head_class;
   return launch_status(s2::launch_adjacency(p, cls, format, out, static_cast<cudaStream_t>(stream)), "adjacency");
+}
+
+int s2attn_debug_adjacency(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class, int format,
+                           void* out, void* stream) {
+  return adjacency_impl(N, G, n_valid, variant, head_class, nullptr, format, out, stream);
+}
+
+int s2attn_debug_adjacency_docs(int64_t N, int64_t G, int64_t n_valid, int variant, int head_class,
+                                const int32_t* doc_bounds, int format, void* out, void* stream) {
+  if (!doc_bounds) return fail(S2_ERR_INVALID_ARG, "null doc_bounds (use s2attn_debug_adjacency without documents)");
+  if (reinterpret_cast<uintptr_t>(doc_bounds) & 7u) return fail(S2_ERR_INVALID_ARG, "doc_bounds must be 8-byte aligned");
+  return adjacency_impl(N, G, n_valid, variant, head_class, doc_bounds, format, out, stream);
 }
 
 int s2attn_debug_wait_probe(int64_t budget_cycles, void* stream) {

@@ -64,6 +64,12 @@ WORKLOADS = {
     "long_n32768_g8192": Workload(
         "long_n32768_g8192", B=1, N=32768, H=32, D=128, G=8192, sharpen_k=True,
         description="B=1 H=32 D=128 N=32768 G=8192, strict, K x2 on 5% of positions"),
+    # the long-context workload with 8 of its 32 heads: the same per-head work,
+    # a quarter of the device memory (about 2.7 GB with the stored dS), for
+    # hardware-counter captures whose per-launch bytes scale by 32 / 8
+    "long_n32768_g8192_h8": Workload(
+        "long_n32768_g8192_h8", B=1, N=32768, H=8, D=128, G=8192, sharpen_k=True,
+        description="B=1 H=8 D=128 N=32768 G=8192, strict, K x2 on 5% of positions (counter captures)"),
     "sweep_n12288_g6144": Workload("sweep_n12288_g6144", B=2, N=12288, H=32, D=128, G=6144),
     "sweep_n12288_g3072": Workload("sweep_n12288_g3072", B=2, N=12288, H=32, D=128, G=3072),
     "sweep_n12288_g2048": Workload("sweep_n12288_g2048", B=2, N=12288, H=32, D=128, G=2048),

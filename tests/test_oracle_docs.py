@@ -122,3 +122,32 @@ def test_document_mask_applies_to_both_head_classes_and_the_window_entry():
     lse = full["lse"][0, H - 1, 6]
     qk = float((x["q"][0, 6, H - 1].double() @ x["k"][0, 6, H - 1].double()) / math.sqrt(D))
     assert abs(lse - qk) < 1e-12
+
+
+@pytest.mark.parametrize("variant,cls", [(STRICT, 0), (STRICT, 1), (ROLLED, 1), (DENSE, 0)])
+def test_adjacency_with_documents(variant, cls):
+    """The document-masked matrix, pinned three ways: one document is no mask;
+    one document per position leaves only the valid diagonal; documents laid
+    out back to back give, for class 0 and the dense graph, causal triangles
+    over the cuts of documents and groups, checked cell by cell."""
+    N, G = 32, 8
+    for nv in (N, 27):
+        A = oracle.adjacency(N, G, nv, variant, cls)
+        one = oracle.adjacency_docs(N, G, nv, variant, cls, np.zeros(N, dtype=np.int32))
+        np.testing.assert_array_equal(one, A)
+        single = oracle.adjacency_docs(N, G, nv, variant, cls, np.arange(N, dtype=np.int32))
+        np.testing.assert_array_equal(single, np.diag(np.arange(N) < nv))
+    lengths = [5, 3, 9, 8, 7]
+    doc = _runs(lengths)
+    got = oracle.adjacency_docs(N, G, N, variant, cls, doc)
+    assert got.sum() == oracle.pair_count_docs(N, G, N, variant, cls, doc)
+    for i in range(N):
+        np.testing.assert_array_equal(oracle.adjacency_row_docs(N, G, N, variant, cls, doc, i), got[i])
+    if variant == DENSE or cls == 0:
+        bounds = np.cumsum([0] + lengths)
+        cuts = sorted(set(bounds.tolist()) | (set() if variant == DENSE else set(range(0, N + 1, G))))
+        expect = np.zeros((N, N), dtype=bool)
+        for a, b in zip(cuts, cuts[1:]):
+            for i in range(a, b):
+                expect[i, a:i + 1] = True
+        np.testing.assert_array_equal(got, expect)
