@@ -634,7 +634,8 @@ def run_ours(args, rank, world, local_rank):
     # CPU oracle leg (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.doc_len:
-        cpu = cpu_baseline_line(oracle_sample({n: x[n] for n in x}, w, variant, 256))
+        # 640 rows of every head: about 15 s of oracle work on the long workload
+        cpu = cpu_baseline_line(oracle_sample({n: x[n] for n in x}, w, variant, min(640, w.G)))
 
     if rank != 0:
         return
