@@ -556,10 +556,13 @@ def run_ours(args, rank, world, local_rank):
     # dk, dv) device -> host.  The copies run on their own streams against two sets
     # of device buffers, so step i's results travel back while step i + 1 computes
     # and step i + 2's inputs arrive (the two directions of the link run at once);
-    # the timed region spans the first input copy to the last result copy.
+    # the forward starts once q, k, v have landed (dout's copy overlaps it) and o
+    # leaves right after the forward.  The timed region spans the first input copy
+    # to the last result copy; 16 steps keep the pipeline's fill and drain (one
+    # input copy, one step, one result copy) a small part of it.
     e2e = None
     if not args.no_e2e:
-        e_steps = max(2, min(args.steps, 6))
+        e_steps = max(2, min(args.steps, 16))
         names_in, names_out = ("q", "k", "v", "dout"), ("o", "dq", "dk", "dv")
         host_in = {n: t.cpu().pin_memory() for n, t in (("q", q), ("k", k), ("v", v), ("dout", do))}
         host_out = [{n: torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for n in names_out} for _ in range(2)]
@@ -573,7 +576,9 @@ def run_ours(args, rank, world, local_rank):
             d["dq"], d["dk"], d["dv"] = (tuple(torch.empty_like(q) for _ in range(3)) if b else grads)
             bufs.append(d)
         s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_qkv = [torch.cuda.Event() for _ in range(2)]
         ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_fwd = [torch.cuda.Event() for _ in range(2)]
         ev_done = [torch.cuda.Event() for _ in range(2)]
         ev_read = [torch.cuda.Event() for _ in range(2)]
         for e in ev_done + ev_read:
@@ -584,22 +589,29 @@ def run_ours(args, rank, world, local_rank):
             d = bufs[b]
             s_in.wait_event(ev_done[b])  # step i - 2 no longer reads this buffer set
             with torch.cuda.stream(s_in):
-                for n in names_in:
+                for n in ("q", "k", "v"):
                     d[n].copy_(host_in[n], non_blocking=True)
+                ev_qkv[b].record(s_in)
+                d["dout"].copy_(host_in["dout"], non_blocking=True)
                 ev_in[b].record(s_in)
-            stream.wait_event(ev_in[b])
+            stream.wait_event(ev_qkv[b])
             stream.wait_event(ev_read[b])  # step i - 2's results have left this buffer set
             qi, ki = d["q"], d["k"]
             if args.rope:
                 s2.rope(d["q"], d["k"], positions, scale=0.25, out=(d["q_in"], d["k_in"]))
                 qi, ki = d["q_in"], d["k_in"]
             s2.forward(qi, ki, d["v"], G, variant, nv, out=d["o"], lse=d["lse"], docs=docs)
+            ev_fwd[b].record(stream)
+            stream.wait_event(ev_in[b])
             s2.backward(qi, ki, d["v"], d["o"], d["dout"], d["lse"], G, variant, nv, grads=(d["dq"], d["dk"], d["dv"]),
                         workspace=ws, docs=docs, stored_ds=stored)
             ev_done[b].record(stream)
+            s_out.wait_event(ev_fwd[b])
+            with torch.cuda.stream(s_out):
+                host_out[b]["o"].copy_(d["o"], non_blocking=True)
             s_out.wait_event(ev_done[b])
             with torch.cuda.stream(s_out):
-                for n in names_out:
+                for n in ("dq", "dk", "dv"):
                     host_out[b][n].copy_(d[n], non_blocking=True)
                 ev_read[b].record(s_out)
 
