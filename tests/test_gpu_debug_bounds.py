@@ -9,7 +9,8 @@ access is skipped and the kernel gives up without a trap.
 
 Checked here: the small parity cases of the other GPU tests (forward, both
 backward forms, padding, one-group sequences, document masks, the emulated
-sequence-parallel ranks, the plain entry points without n_valid) run through
+sequence-parallel ranks, the plain entry points without n_valid) and 32
+seeded random shapes run through
 the debug build with no violation recorded, give results bit for bit equal to
 the normal build's, and match the float64 oracle.  The recording path itself
 is exercised by the probe entry point, which runs the same check on a chosen
@@ -171,3 +172,24 @@ def test_probe_records_the_first_violation_without_a_fault():
         torch.cuda.synchronize()
         _no_violation()
         assert torch.isfinite(o).all()
+
+
+@pytest.mark.parametrize("seed", range(100, 132))
+def test_debug_build_on_random_shapes(seed):
+    """Seeded random shapes, padding and document cuts (the fuzz test's generator,
+    other seeds) through the debug build: no violation, bitwise the normal
+    build's results, and the oracle's within the parity tolerances."""
+    from tests.test_gpu_fuzz import _case
+
+    B, N, H, D, G, variant, nv, ids = _case(seed)
+    where = str((seed, B, N, H, D, G, variant, nv, ids is not None))
+    x = synthetic.draw(B, N, H, D, seed=9000 + seed)
+    docs = s2.doc_bounds(torch.from_numpy(ids).cuda()) if ids is not None else None
+    r = _debug_and_release(x, G, variant, nv, docs)
+    ref = oracle.attention(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, n_valid=nv, doc=ids)
+    n = N if nv is None else nv
+    check_o(r["o"][:, :n], ref["o"][:, :n], where)
+    check_lse(r["lse"].cpu().numpy(), ref["lse"], where)
+    for name in ("dq", "dk", "dv"):
+        check_grad(name, to_np(r[name])[:, :n], ref[name][:, :n], where)
+        check_grad(name, to_np(r[name + "_ds"])[:, :n], ref[name][:, :n], where + " stored dS")

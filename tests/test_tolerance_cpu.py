@@ -2,6 +2,8 @@
 the scale rule of the gradient check."""
 from __future__ import annotations
 
+import math
+
 import numpy as np
 import pytest
 import torch
@@ -50,3 +52,22 @@ def test_gradient_scale_comes_from_the_given_oracle_maximum():
     tolerance.check_grad("dv", ref + 0.05, ref, "sample", ref_max=100.0)
     with pytest.raises(AssertionError):
         tolerance.check_grad("dv", ref + 0.05, ref, "sample")
+
+
+def test_lse_bound_covers_the_rounded_row_sum_and_is_nearly_tight():
+    """The lse tolerance is the worst case of summing bf16-rounded weights:
+    random rows of few keys stay inside it, and weights placed just above a
+    power of two (each rounded down by almost 2^-8 of its value) come within a
+    few percent of it."""
+    rng = np.random.default_rng(5)
+    worst = 0.0
+    for n in (2, 3, 4, 8, 64):
+        z = rng.normal(size=(20000, n)) * 3
+        p = np.exp2(z - z.max(axis=1, keepdims=True) + rng.uniform(0, 8, size=(20000, 1)))  # lazy max: p up to 2^8
+        l, lt = p.sum(axis=1), tolerance.bf16_rne(p).sum(axis=1)
+        worst = max(worst, float(np.abs(np.log(lt) - np.log(l)).max()))
+    assert worst <= tolerance.LSE_ABS
+    # adversarial: every weight just above a power of two, one ulp-half minus a hair
+    p = np.ldexp(1.0 + 2.0 ** -8 - 2.0 ** -20, rng.integers(-8, 8, size=16))
+    gap = abs(np.log(tolerance.bf16_rne(p).sum()) - np.log(p.sum()))
+    assert 0.95 * math.log1p(2.0 ** -8) < gap <= tolerance.LSE_ABS

@@ -16,6 +16,7 @@ computed, never a value read from the CUDA output.
 from __future__ import annotations
 
 import json
+import math
 import os
 
 import numpy as np
@@ -23,7 +24,14 @@ import torch
 
 O_MAX, O_MEAN = 1e-2, 1e-3
 G_MAX, G_MEAN = 1e-2, 1e-3
-LSE_ABS = 2e-3
+# lse has no stated tolerance; this one follows from the kernel's arithmetic.  The
+# forward's row sum l adds the softmax weights after their rounding to bf16 (so
+# that o stays a convex combination of the v_j), and round-to-nearest-even to
+# bf16's 8 significant bits changes each weight by at most 2^-8 of its value.  A
+# sum of such weights is off by at most 2^-8 relative, so ln l by at most
+# ln(1 + 2^-8) = 3.90e-3; the fp32 scores (D bf16 products accumulated in fp32,
+# times 1/sqrt(D)) and the approximate exp2 / log2 add well under 1e-4.
+LSE_ABS = math.log1p(2.0 ** -8) + 1e-4
 
 # One record per check_o call: the test it ran in (set by an autouse fixture in
 # conftest.py), where, the errors, the storage floor and how many elements passed
