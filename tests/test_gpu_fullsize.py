@@ -200,3 +200,50 @@ def test_group_ratio_sweep_full_causal(stored):
 @PATHS
 def test_ragged_tail_n100000(stored):
     _check_workload("ragged_n100000_g8192", 0, stored)
+
+
+def test_tensors_beyond_2_31_elements():
+    """Maximum sizes: B1 N131072 H132 D128 G8192, 2.2e9 elements (4.4 GB) per
+    tensor, so any element offset kept in 32 bits would wrap.  The forward and
+    the recomputing backward (the stored dS would need about 140 GB here) run
+    through the C ABI; the oracle checks windows of the first and last heads of
+    each class at the start, in the middle and at the end of the sequence, where
+    the offsets are largest."""
+    B, N, H, D, G, variant = 1, 131072, 132, 128, 8192, 0
+    assert B * N * H * D > 2 ** 31
+    x = synthetic.draw(B, N, H, D, seed=31)
+    dev = {n: t.cuda() for n, t in x.items()}
+    o, lse = s2.forward(dev["q"], dev["k"], dev["v"], G, variant)
+    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, G, variant)
+    torch.cuda.synchronize()
+    s2.check_status()
+    for name, t in (("o", o), ("dq", dq), ("dk", dk), ("dv", dv)):
+        assert bool(torch.isfinite(t).all()), name
+    s = G // 2
+    heads = (0, H // 2 - 1, H // 2, H - 1)
+    # class-0 segment ends at multiples of G; class-1 (strict) at s + kG and at N
+    windows = [(0, W, False), (N // 2 - W, N // 2, True), (N // 2 + s - W, N // 2 + s, True), (N - W, N, True)]
+    jobs, ref_max = [], {"dq": 0.0, "dk": 0.0, "dv": 0.0}
+    for r0, r1, at_end in windows:
+        ref = oracle.attention_window(x["q"], x["k"], x["v"], x["dout"], G=G, variant=variant, rows=(r0, r1),
+                                      heads=list(heads))
+        jobs.append((r0, r1, at_end, ref))
+        ref_max["dq"] = max(ref_max["dq"], float(np.abs(ref["dq"]).max()))
+        for t, h in enumerate(heads):
+            cls = int(h >= H // 2)
+            seg_end = (r1 % G == 0) if cls == 0 else (r1 == N or (r1 - s) % G == 0)
+            if at_end and seg_end:
+                for n in ("dk", "dv"):
+                    ref_max[n] = max(ref_max[n], float(np.abs(ref[n][t]).max()))
+    assert all(v > 0 for v in ref_max.values()), ref_max
+    for r0, r1, at_end, ref in jobs:
+        for t, h in enumerate(heads):
+            where = "N131072 H132 head %d rows [%d, %d)" % (h, r0, r1)
+            check_o(o[0, r0:r1, h], ref["o"][t], where)
+            check_lse(lse[0, h, r0:r1], ref["lse"][t], where)
+            check_grad("dq", to_np(dq[0, r0:r1, h]), ref["dq"][t], where, ref_max["dq"])
+            cls = int(h >= H // 2)
+            seg_end = (r1 % G == 0) if cls == 0 else (r1 == N or (r1 - s) % G == 0)
+            if at_end and seg_end:  # every query that sees these keys lies in the window
+                for n, g in (("dk", dk), ("dv", dv)):
+                    check_grad(n, to_np(g[0, r0:r1, h]), ref[n][t], where, ref_max[n])
