@@ -547,7 +547,7 @@ def run_ours(args, rank, world, local_rank):
         (("rope", 5, 0),) if args.rope else ())
     samples = {name: [e[a].elapsed_time(e[b]) for e in evs] for name, a, b in stages}
     per = {name: sum(t) / args.steps for name, t in samples.items()}
-    # this rank's spread over the timed steps (the survey's protocol: median and minimum per pass)
+    # this rank's spread over the timed steps: median and minimum per pass
     per_spread = {name: {"median": statistics.median(t), "min": min(t)} for name, t in samples.items()}
     clocks = clk.summary()
 
