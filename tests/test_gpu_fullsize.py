@@ -247,3 +247,44 @@ def test_tensors_beyond_2_31_elements():
             if at_end and seg_end:  # every query that sees these keys lies in the window
                 for n, g in (("dk", dk), ("dv", dv)):
                     check_grad(n, to_np(g[0, r0:r1, h]), ref[n][t], where, ref_max[n])
+
+
+@PATHS
+def test_long_context_packed_documents(stored):
+    """The long-context workload packed with documents of 4096 tokens (the step
+    bench.py --doc-len 4096 times), both backward forms, against the oracle under
+    the same document mask: windows at document starts (o, lse, dq) and at
+    document ends, where every query that sees the window's keys lies in the
+    window (dk, dv complete as well)."""
+    name, doc_len = "long_n32768_g8192", 4096
+    w = synthetic.WORKLOADS[name]
+    x = _inputs(w.B, w.N, w.H, w.D, w.seed, w.sharpen_k)
+    ids = np.ascontiguousarray(np.broadcast_to((np.arange(w.N) // doc_len).astype(np.int32), (w.B, w.N)))
+    dev = {n: t.cuda() for n, t in x.items()}
+    docs = s2.doc_bounds(torch.from_numpy(ids).cuda())
+    o, lse = s2.forward(dev["q"], dev["k"], dev["v"], w.G, 0, docs=docs)
+    dq, dk, dv = s2.backward(dev["q"], dev["k"], dev["v"], o, dev["dout"], lse, w.G, 0, docs=docs, stored_ds=stored)
+    torch.cuda.synchronize()
+    s2.check_status()
+    H = w.H
+    heads = (0, H // 2 - 1, H // 2, H - 1)
+    windows = [(0, W, False), (3 * doc_len, 3 * doc_len + W, False), (2 * doc_len - W, 2 * doc_len, True),
+               (5 * doc_len - W, 5 * doc_len, True), (w.N - W, w.N, True)]
+    jobs, ref_max = [], {"dq": 0.0, "dk": 0.0, "dv": 0.0}
+    for r0, r1, at_end in windows:
+        ref = oracle.attention_window(x["q"], x["k"], x["v"], x["dout"], G=w.G, variant=0, rows=(r0, r1),
+                                      heads=list(heads), doc=ids)
+        jobs.append((r0, r1, at_end, ref))
+        ref_max["dq"] = max(ref_max["dq"], float(np.abs(ref["dq"]).max()))
+        if at_end:
+            for n in ("dk", "dv"):
+                ref_max[n] = max(ref_max[n], float(np.abs(ref[n]).max()))
+    for r0, r1, at_end, ref in jobs:
+        for t, h in enumerate(heads):
+            where = "%s documents of %d head %d rows [%d, %d)" % (name, doc_len, h, r0, r1)
+            check_o(o[0, r0:r1, h], ref["o"][t], where)
+            check_lse(lse[0, h, r0:r1], ref["lse"][t], where)
+            check_grad("dq", to_np(dq[0, r0:r1, h]), ref["dq"][t], where, ref_max["dq"])
+            if at_end:
+                for n, g in (("dk", dk), ("dv", dv)):
+                    check_grad(n, to_np(g[0, r0:r1, h]), ref[n][t], where, ref_max[n])
