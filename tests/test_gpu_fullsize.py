@@ -259,7 +259,7 @@ def test_long_context_packed_documents(stored):
     name, doc_len = "long_n32768_g8192", 4096
     w = synthetic.WORKLOADS[name]
     x = _inputs(w.B, w.N, w.H, w.D, w.seed, w.sharpen_k)
-    ids = np.ascontiguousarray(np.broadcast_to((np.arange(w.N) // doc_len).astype(np.int32), (w.B, w.N)))
+    ids = np.tile((np.arange(w.N) // doc_len).astype(np.int32), (w.B, 1))
     dev = {n: t.cuda() for n, t in x.items()}
     docs = s2.doc_bounds(torch.from_numpy(ids).cuda())
     o, lse = s2.forward(dev["q"], dev["k"], dev["v"], w.G, 0, docs=docs)
