@@ -404,8 +404,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       // P of the current tile as bf16 pairs, from its exponentials to its dS: dS uses
       // the same rounded P as dV += P^T dO
       uint32_t pk[32];
-      // P(nn): S^T -> P^T (bf16 pairs into R1 and pk); both 32-column loads are in
-      // flight before the one wait
+      // P(nn): S^T -> P^T (bf16 pairs into R1 and pk); the row's 64 columns in one load
       auto p_step = [&](int nn, int qtile) -> bool {
         const int sq = nn % kQSlots;
         // masks on the diagonal tile, on a key tile with padding and under a
@@ -418,8 +417,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_after();
         const float2* nl = reinterpret_cast<const float2*>(smem + L::kLse + sq * L::kRowBytes) + 32 * x;
         uint32_t sv[64];
-        tmem_ld32(tR1 + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tR1 + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld64(tR1 + lane_off + 64 * x, sv);
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -434,8 +432,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           pk[i] = pack_bf16(p0, p1);
         }
         // P^T pairs over the S columns [64x, 64x + 32), all read already
-        tmem_st16(tR1 + lane_off + 64 * x, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-        tmem_st16(tR1 + lane_off + 64 * x + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+        tmem_st32(tR1 + lane_off + 64 * x, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(P_READY));
@@ -466,8 +463,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         tc_fence_after();
         const float2* nd = reinterpret_cast<const float2*>(smem + L::kDelta + sd * L::kRowBytes) + 32 * x;
         uint32_t dp[64];
-        tmem_ld32(tR2 + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tR2 + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_ld64(tR2 + lane_off + 64 * x, dp);
         tmem_wait_ld();
         uint32_t keep[32];  // this row's dS pairs (also stored after the hand-off)
 #pragma unroll
@@ -477,8 +473,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           const float2 ds = __fmul2_rn(pv, d2);
           keep[i] = pack_bf16(ds.x, ds.y);
         }
-        tmem_st16(tR2 + lane_off + 64 * x, *reinterpret_cast<const uint32_t(*)[16]>(&keep[0]));
-        tmem_st16(tR2 + lane_off + 64 * x + 16, *reinterpret_cast<const uint32_t(*)[16]>(&keep[16]));
+        tmem_st32(tR2 + lane_off + 64 * x, keep);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(DS_READY));
@@ -786,11 +781,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         ok = s2_wait(bar(S_FULL + (jj % 2)), (jj / 2) & 1, abort_flag, status, 4);
         if (!ok) break;
         tc_fence_after();
-        // both 32-column loads in flight before one wait; P kept as the bf16 pairs
+        // the row's 64 columns in one load; P kept as the bf16 pairs
         // dS is formed from (the same rounding as the dK/dV pass)
         uint32_t sv[64];
-        tmem_ld32(tS + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(tS + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+        tmem_ld64(tS + lane_off + 64 * x, sv);
         tmem_wait_ld();
         uint32_t pk[32];
 #pragma unroll
@@ -808,8 +802,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         if (!ok) break;
         tc_fence_after();
         uint32_t dp[64];
-        tmem_ld32(tDP + lane_off + 64 * x, *reinterpret_cast<uint32_t(*)[32]>(&dp[0]));
-        tmem_ld32(tDP + lane_off + 64 * x + 32, *reinterpret_cast<uint32_t(*)[32]>(&dp[32]));
+        tmem_ld64(tDP + lane_off + 64 * x, dp);
         tmem_wait_ld();
         uint32_t dsp[32];
 #pragma unroll
@@ -820,8 +813,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           dsp[i] = pack_bf16(ds.x, ds.y);
         }
         // dS pairs of key columns [64x, 64x + 64) -> S columns 64x + [0, 32), already read
-        tmem_st16(tS + lane_off + 64 * x, *reinterpret_cast<const uint32_t(*)[16]>(&dsp[0]));
-        tmem_st16(tS + lane_off + 64 * x + 16, *reinterpret_cast<const uint32_t(*)[16]>(&dsp[16]));
+        tmem_st32(tS + lane_off + 64 * x, dsp);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(DS_READY));

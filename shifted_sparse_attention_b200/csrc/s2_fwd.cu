@@ -332,8 +332,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
           if (!ok) break;
           tc_fence_after();
           uint32_t s[kTile];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) tmem_ld32(tS + j * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[j * 32]));
+          tmem_ld128(tS, s);
           tmem_wait_ld();
 
           // Masks (the causal triangle of the diagonal tile, padded keys or rows,
@@ -401,8 +400,7 @@ __global__ void __launch_bounds__(fwd::kThreads, 1)
             }
           }
           // P (bf16 pairs) -> TMEM columns [0, 64) of S_x, the A operand of O_x += P_x V
-          tmem_st32(tS, *reinterpret_cast<const uint32_t(*)[32]>(&s[0]));
-          tmem_st32(tS + 32, *reinterpret_cast<const uint32_t(*)[32]>(&s[32]));
+          tmem_st64(tS, *reinterpret_cast<const uint32_t(*)[64]>(&s[0]));
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(P_FULL + x));
