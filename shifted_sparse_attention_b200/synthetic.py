@@ -70,6 +70,10 @@ WORKLOADS = {
     "long_n32768_g8192_h8": Workload(
         "long_n32768_g8192_h8", B=1, N=32768, H=8, D=128, G=8192, sharpen_k=True,
         description="B=1 H=8 D=128 N=32768 G=8192, strict, K x2 on 5% of positions (counter captures)"),
+    # the long-context workload at head dimension 64 (the kernels' other D)
+    "long_n32768_g8192_d64": Workload(
+        "long_n32768_g8192_d64", B=1, N=32768, H=32, D=64, G=8192, sharpen_k=True,
+        description="B=1 H=32 D=64 N=32768 G=8192, strict, K x2 on 5% of positions"),
     "sweep_n12288_g6144": Workload("sweep_n12288_g6144", B=2, N=12288, H=32, D=128, G=6144),
     "sweep_n12288_g3072": Workload("sweep_n12288_g3072", B=2, N=12288, H=32, D=128, G=3072),
     "sweep_n12288_g2048": Workload("sweep_n12288_g2048", B=2, N=12288, H=32, D=128, G=2048),

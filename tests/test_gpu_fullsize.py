@@ -186,6 +186,11 @@ def test_long_context_n32768_g8192(stored):
 
 
 @PATHS
+def test_long_context_head_dim_64(stored):
+    _check_workload("long_n32768_g8192_d64", 0, stored)
+
+
+@PATHS
 @pytest.mark.parametrize("name", ["sweep_n12288_g6144", "sweep_n12288_g3072", "sweep_n12288_g2048",
                                   "sweep_n12288_g1536"])
 def test_group_ratio_sweep(name, stored):
